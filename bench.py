@@ -1,0 +1,467 @@
+#!/usr/bin/env python
+"""Benchmark of the fused chunked top-K KL distillation loss on B200.
+
+One step = the whole hot path over one batch of synthetic input:
+  top-K cache build of the batch's teacher logits [T, V] (bf16)
+  -> fused chunked KL forward (loss, lse) -> fused chunked KL backward (dH, dW),
+with the cache the build produced feeding the loss.
+
+Default workload: the toy output head at 32K tokens (T=32768, d=4096,
+V=131072, K=100, chunk=2048, bf16 operands, fp32 accumulation).
+
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+
+Prints ONE JSON line (rank 0).  Multi-GPU runs are independent replicas (weak
+scaling, no collective on the data path); time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "tokens/s & TFLOP/s (8TdV) fused top-K KL fwd+bwd; % BF16 tensor peak; peak mem"
+UNIT = "tokens/s"
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="kd", choices=["kd", "reference"])
+    ap.add_argument("--workload", default="head-32k")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=0, help="oracle rows per CPU step (0 = auto)")
+    ap.add_argument("--sweep-memory", action="store_true",
+                    help="print the peak-memory vs T sweep instead of the bench line")
+    return ap.parse_args()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def _workload(name):
+    from chunked_kl_loss_chunk_b200 import inputs
+    return dict(inputs.WORKLOADS[name])
+
+
+def _config(w, name, extra=None):
+    c = {"workload": name, "T": w["T"], "d": w["d"], "V": w["V"], "K": w["K"],
+         "chunk": w["chunk"], "temperature": 1.0,
+         "step": "top-K cache build of teacher logits [T,V] + fused fwd + fused bwd (dH, dW)",
+         "l2": "inputs larger than L2 (W and teacher logits exceed 126 MB); no flush"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def _cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def _cpu_sample_step(W64, h_rows, logits_rows, K, tau=1.0):
+    """One bounded sample of the step on the host cores with the fp64 oracle."""
+    import oracle
+    vals, idx = oracle.topk_rows(logits_rows, K)
+    _, lse, _ = oracle.forward(h_rows, W64, vals, idx, tau)
+    oracle.backward(h_rows, W64, vals, idx, tau)
+
+
+def _cpu_setup(w, rows, seed=0):
+    import numpy as np
+    import torch
+    import oracle
+    from chunked_kl_loss_chunk_b200 import inputs
+    # The same distributions as the GPU arm, drawn on the host.
+    g = torch.Generator().manual_seed(seed * 1000 + 1)
+    W = (torch.randn((w["V"], w["d"]), generator=g) / math.sqrt(w["d"])).to(torch.bfloat16)
+    Wn = W.view(torch.int16).numpy().view(np.uint16)
+    W64 = oracle.bf16_bits_to_f64(Wn)
+    h, _, _, _ = inputs.make_loss_inputs(rows, w["d"], 8, 1, dtype=torch.bfloat16, seed=seed)
+    hn = h.view(torch.int16).numpy().view(np.uint16)
+    x = inputs.make_teacher_logits(rows, w["V"], seed=seed)
+    xn = x.view(torch.int16).numpy().view(np.uint16)
+    return W64, hn, xn
+
+
+def cpu_baseline(w, rows=0, steps=1):
+    """Oracle tokens/s on a bounded sample (rows positions per step)."""
+    if rows <= 0:
+        rows = 16
+    W64, hn, xn = _cpu_setup(w, rows)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        _cpu_sample_step(W64, hn, xn, w["K"])
+    dt = time.perf_counter() - t0
+    return {"value": rows * steps / dt, "unit": UNIT, "cores": _cpu_threads(), "kind": "oracle",
+            "sample": f"{rows} positions x {steps} step(s) of the {w['T']}-position batch: "
+                      f"fp64 top-K (full stable sort of V={w['V']}), forward and backward "
+                      f"(d={w['d']}); {dt:.2f} s"}
+
+
+def run_reference(args, rank):
+    """Reference arm: the fp64 CPU oracle as it stands, rank 0 only."""
+    if rank != 0:
+        return
+    w = _workload(args.workload)
+    rows = args.cpu_rows or 8
+    W64, hn, xn = _cpu_setup(w, rows)
+    for _ in range(args.warmup):
+        _cpu_sample_step(W64, hn, xn, w["K"])
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        _cpu_sample_step(W64, hn, xn, w["K"])
+    dt = time.perf_counter() - t0
+    v = rows * args.steps / dt
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1000 * dt / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(w, args.workload, {"sample_rows_per_step": rows}),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": _cpu_threads(), "kind": "oracle",
+                             "sample": f"{rows} positions per step (top-K, forward, backward) of "
+                                       f"the {w['T']}-position workload"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    def __init__(self, dev_index):
+        self.proc = None
+        self.path = None
+        self.dev = dev_index
+
+    def start(self):
+        import torch
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        ident = str(self.dev)
+        try:
+            u = torch.cuda.get_device_properties(self.dev).uuid
+            ident = "GPU-" + str(u) if not str(u).startswith("GPU-") else str(u)
+        except Exception:
+            pass
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={ident}", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in open(self.path):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_kd(args, rank, world):
+    import torch
+    import torch.distributed as dist
+    from chunked_kl_loss_chunk_b200 import build as kbuild
+    from chunked_kl_loss_chunk_b200 import inputs, kd
+
+    kbuild.build()
+    kd.load()
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = _workload(args.workload)
+    T, d, V, K, chunk = w["T"], w["d"], w["V"], w["K"], w["chunk"]
+    dt = torch.bfloat16 if w["dtype"] == "bf16" else torch.float32
+
+    # inputs of this rank's replica (seeded by rank)
+    h, W, _, _ = inputs.make_loss_inputs(T, d, V, 1, dtype=dt, seed=rank, device=dev)
+    logits = inputs.make_teacher_logits(T, V, seed=rank, device=dev)
+    vals = torch.empty((T, K), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, K), dtype=torch.int32, device=dev)
+    ws_topk = kd.alloc_workspace(kd.kd_topk_workspace_size(T, V, K), dev)
+    ws = kd.workspace_for(h, W, K, chunk)
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    lse = torch.empty((T,), dtype=torch.float32, device=dev)
+    dH = torch.empty_like(h)
+    dW = torch.empty((V, d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    sp = stream.cuda_stream
+    code = kd.KD_DTYPE_BF16 if dt == torch.bfloat16 else kd.KD_DTYPE_F32
+    ev_topk = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev_fwd = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def step(timing=None):
+        if timing is not None:
+            ev_topk[0].record()
+        st = kd.kd_topk_build(logits.data_ptr(), kd.KD_DTYPE_BF16, T, V, K, vals.data_ptr(),
+                              idx.data_ptr(), ws_topk.data_ptr(), ws_topk.numel(), sp)
+        if timing is not None:
+            ev_topk[1].record()
+        st |= kd.kd_fused_kl_fwd(h.data_ptr(), W.data_ptr(), code, T, d, V, vals.data_ptr(),
+                                 idx.data_ptr(), K, chunk, 1.0, loss.data_ptr(), lse.data_ptr(),
+                                 None, ws.data_ptr(), ws.numel(), sp)
+        if timing is not None:
+            ev_fwd[1].record()
+        st |= kd.kd_fused_kl_bwd(h.data_ptr(), W.data_ptr(), code, T, d, V, vals.data_ptr(),
+                                 idx.data_ptr(), K, chunk, 1.0, lse.data_ptr(), None, dH.data_ptr(),
+                                 dW.data_ptr(), 0, ws.data_ptr(), ws.numel(), sp)
+        if st != 0:
+            raise RuntimeError(f"libkd call failed ({st})")
+        if timing is not None:
+            torch.cuda.synchronize()
+            timing["topk_ms"].append(ev_topk[0].elapsed_time(ev_topk[1]))
+            timing["fwd_ms"].append(ev_topk[1].elapsed_time(ev_fwd[1]))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # warm-up
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert kd.read_device_status(ws) == kd.KD_OK
+
+    # component timings (separate, untimed-region passes)
+    comp = {"topk_ms": [], "fwd_ms": []}
+    for _ in range(2):
+        step(comp)
+
+    prof = kd.GemmProfiler(capacity=4 * ((T + chunk - 1) // chunk) * args.steps + 16)
+    sampler = ClockSampler(local) if rank == 0 else None
+    torch.cuda.reset_peak_memory_stats(dev)
+    barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    n0 = kd.kd_launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with prof:
+        e0.record()
+        for _ in range(args.steps):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+    n_launch = kd.kd_launch_count() - n0
+    clocks = sampler.stop() if sampler else None
+    barrier()
+    ms_total = e0.elapsed_time(e1)
+    peak_bytes = torch.cuda.max_memory_allocated(dev)
+    if world > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    tokens = T * args.steps * world
+    value = tokens / (ms_total / 1000.0)
+    flop_step = 8.0 * T * d * V
+
+    # per-GEMM-kind breakdown from the live events
+    res = prof.results()
+    kinds = {}
+    for k, f, ms in res:
+        e = kinds.setdefault(kd.GEMM_KIND_NAMES[k], {"launches": 0, "ms": 0.0, "flops": 0.0})
+        e["launches"] += 1
+        e["ms"] += ms
+        e["flops"] += f
+    dom = max(kinds.items(), key=lambda kv: kv[1]["ms"])
+    peaks, peak_src = _peaks()
+    peak_sus = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    achieved = dom[1]["flops"] / (dom[1]["ms"] / 1000.0) / 1e12
+    gemm_ms_step = sum(v["ms"] for v in kinds.values()) / args.steps
+    topk_ms = statistics.median(comp["topk_ms"])
+    fwd_ms = statistics.median(comp["fwd_ms"])
+    loss_ms = ms_step - topk_ms
+    loss_tflops = flop_step / (loss_ms / 1000.0) / 1e12
+
+    # loss-path memory: what the fused loss holds (inputs, cache, outputs, workspace)
+    loss_path_bytes = (h.numel() * h.element_size() + W.numel() * W.element_size()
+                       + vals.numel() * 4 + idx.numel() * 4 + lse.numel() * 4
+                       + dH.numel() * dH.element_size() + dW.numel() * 4 + ws.numel())
+
+    # e2e: host-resident inputs through the same public API, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        h_host = h.cpu().pin_memory()
+        W_host = W.cpu().pin_memory()
+        x_host = logits.cpu().pin_memory()
+        loss_host = torch.empty((), dtype=torch.float32).pin_memory()
+        h2d = h.numel() * h.element_size() + W.numel() * W.element_size() + x_host.numel() * 2
+
+        def e2e_step():
+            h.copy_(h_host, non_blocking=True)
+            W.copy_(W_host, non_blocking=True)
+            logits.copy_(x_host, non_blocking=True)
+            step()
+            loss_host.copy_(loss, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        ems = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([ems], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": tokens / (ems / 1000.0), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+               "d2h_bytes_per_step": 4, "ms_per_step": ems / args.steps}
+
+    if rank != 0:
+        return
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, rows=args.cpu_rows or 16)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
+        "data": "synthetic",
+        "config": _config(w, args.workload, {"parallelism": f"replicas x{world}"}),
+        "loss_fwd_bwd": {"ms": loss_ms, "tokens_per_s": T / (loss_ms / 1000.0),
+                          "tflops": loss_tflops,
+                          "frac_bf16_peak_sustained": loss_tflops / peak_sus,
+                          "frac_bf16_peak_burst": loss_tflops / float(peaks["bf16_tflops"]),
+                          "fwd_ms": fwd_ms, "bwd_ms": loss_ms - fwd_ms,
+                          "gemm_ms": gemm_ms_step},
+        "topk_build": {"ms": topk_ms, "gbs": (T * V * 2 + T * K * 8) / (topk_ms / 1000.0) / 1e9,
+                       "frac_hbm_peak": (T * V * 2 + T * K * 8) / (topk_ms / 1000.0) / 1e9
+                       / float(peaks["hbm_gbs"])},
+        "gemm_kernels": {k: {"launches": v["launches"], "ms_per_launch": v["ms"] / v["launches"],
+                             "tflops": v["flops"] / (v["ms"] / 1000.0) / 1e12}
+                         for k, v in kinds.items()},
+        "peak_mem_bytes": int(peak_bytes),
+        "loss_path_bytes": int(loss_path_bytes),
+        "dense_logits_grid_bytes_fp32": int(T * V * 4),
+        "roofline": {"bound": "tensor", "kernel": f"gemm_kernel ({dom[0]})",
+                     "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
+                     "frac": achieved / peak_sus, "traffic": None,
+                     "peak_source": f"{peak_src} bf16_tflops_sustained (kernel inside a long step)"},
+        "gpu_launches": int(n_launch),
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def sweep_memory(args):
+    """Peak device memory of the fused loss (fwd + bwd) vs T at d=4096, V=131072."""
+    import torch
+    from chunked_kl_loss_chunk_b200 import build as kbuild
+    from chunked_kl_loss_chunk_b200 import inputs, kd
+    kbuild.build()
+    dev = torch.device("cuda", 0)
+    d, V, K, chunk = 4096, 131072, 100, 4096
+    out = []
+    for T in (4096, 8192, 16384, 32768, 65536, 131072, 262144):
+        torch.cuda.empty_cache()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)
+        h, W, vals, idx = inputs.make_loss_inputs(T, d, V, K, dtype=torch.bfloat16, seed=0, device=dev)
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats(dev)
+        loss, lse, _, ws = kd.fused_kl_fwd(h, W, vals, idx, chunk, 1.0)
+        dH, dW, _ = kd.fused_kl_bwd(h, W, vals, idx, lse, chunk, 1.0, ws=ws)
+        torch.cuda.synchronize()
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        out.append({"T": T, "peak_bytes": int(peak), "dense_grid_fp32_bytes": T * V * 4})
+        del h, W, vals, idx, loss, lse, ws, dH, dW
+    xs = [o["T"] for o in out]
+    ys = [o["peak_bytes"] for o in out]
+    n = len(xs)
+    mx, my = sum(xs) / n, sum(ys) / n
+    b = sum((x - mx) * (y - my) for x, y in zip(xs, ys)) / sum((x - mx) ** 2 for x in xs)
+    a = my - b * mx
+    ss_res = sum((y - (a + b * x)) ** 2 for x, y in zip(xs, ys))
+    ss_tot = sum((y - my) ** 2 for y in ys)
+    print(json.dumps({"sweep": out, "fit": {"intercept_bytes": a, "bytes_per_token": b,
+                                            "r2": 1 - ss_res / ss_tot}}), flush=True)
+
+
+def main():
+    args = _args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    if args.sweep_memory:
+        sweep_memory(args)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        run_kd(args, rank, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

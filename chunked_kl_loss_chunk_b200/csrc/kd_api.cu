@@ -1,0 +1,208 @@
+// kd_api.cu -- the C ABI declared in include/kd.h: argument validation,
+// workspace sizing, device status, and dispatch to the kernels.
+#include <math.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "kd_internal.h"
+
+namespace {
+
+uint64_t g_wait_limit_ns = 4000000000ull;  // 4 s
+std::atomic<uint64_t> g_launches{0};
+
+struct Profile {
+  void* const* start = nullptr;
+  void* const* end = nullptr;
+  int* kinds = nullptr;
+  double* flops = nullptr;
+  int capacity = 0, mask = 0, n = 0;
+  bool armed = false;   // set between profile_before and profile_after
+} g_prof;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int num_sms_current() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+constexpr int KD_MAX_K = 1024;
+
+}  // namespace
+
+namespace kd {
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+void profile_before(int kind, double flops, cudaStream_t s) {
+  g_prof.armed = false;
+  if (!g_prof.start || !(g_prof.mask & kind) || g_prof.n >= g_prof.capacity) return;
+  cudaEventRecord(static_cast<cudaEvent_t>(g_prof.start[g_prof.n]), s);
+  if (g_prof.kinds) g_prof.kinds[g_prof.n] = kind;
+  if (g_prof.flops) g_prof.flops[g_prof.n] = flops;
+  g_prof.armed = true;
+}
+
+void profile_after(cudaStream_t s) {
+  if (!g_prof.armed) return;
+  cudaEventRecord(static_cast<cudaEvent_t>(g_prof.end[g_prof.n]), s);
+  ++g_prof.n;
+  g_prof.armed = false;
+}
+
+}  // namespace kd
+
+extern "C" {
+
+const char* kd_status_string(int status) {
+  switch (status) {
+    case KD_OK: return "KD_OK";
+    case KD_ERR_INVALID_ARG: return "KD_ERR_INVALID_ARG";
+    case KD_ERR_UNSUPPORTED: return "KD_ERR_UNSUPPORTED";
+    case KD_ERR_WORKSPACE: return "KD_ERR_WORKSPACE";
+    case KD_ERR_BAD_INDEX: return "KD_ERR_BAD_INDEX";
+    case KD_ERR_TIMEOUT: return "KD_ERR_TIMEOUT";
+    case KD_ERR_CUDA: return "KD_ERR_CUDA";
+    default: return "KD_ERR_UNKNOWN";
+  }
+}
+
+int kd_version(void) { return (1 << 16) | 0; }
+
+size_t kd_topk_workspace_size(int64_t T, int64_t V, int K) {
+  (void)T;
+  (void)V;
+  (void)K;
+  return 1024;
+}
+
+kd_status kd_topk_build(const void* logits, int dtype, int64_t T, int64_t V, int K,
+                        float* out_vals, int32_t* out_idx, void* ws, size_t ws_bytes,
+                        void* stream) {
+  if (!logits || !out_vals || !out_idx || !ws) return KD_ERR_INVALID_ARG;
+  if (T < 1 || V < 1 || K < 1 || K > V) return KD_ERR_INVALID_ARG;
+  if (!aligned(logits, 16) || !aligned(out_vals, 16) || !aligned(out_idx, 16) ||
+      !aligned(ws, 1024))
+    return KD_ERR_INVALID_ARG;
+  if (dtype != KD_DTYPE_BF16) return KD_ERR_UNSUPPORTED;
+  if (K > KD_MAX_K || V >= (int64_t(1) << 31)) return KD_ERR_UNSUPPORTED;
+  if (ws_bytes < kd_topk_workspace_size(T, V, K)) return KD_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int sms = num_sms_current();
+  if (sms <= 0) return KD_ERR_CUDA;
+  if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return KD_ERR_CUDA;
+  if (kd::launch_topk_bf16(logits, T, V, K, out_vals, out_idx, s, sms) != cudaSuccess)
+    return KD_ERR_CUDA;
+  return KD_OK;
+}
+
+size_t kd_fused_kl_workspace_size(int64_t T, int64_t d, int64_t V, int K, int64_t chunk,
+                                  int dtype) {
+  if (T < 1 || d < 1 || V < 1 || K < 1 || chunk < 1) return 0;
+  return kd::ws_layout(T, d, V, K, chunk, dtype).total;
+}
+
+static kd_status validate_loss(const void* h, const void* W, int dtype, int64_t T, int64_t d,
+                               int64_t V, const float* t_vals, const int32_t* t_idx, int K,
+                               int64_t chunk, float tau, void* ws, size_t ws_bytes) {
+  if (!h || !W || !t_vals || !t_idx || !ws) return KD_ERR_INVALID_ARG;
+  if (T < 1 || d < 1 || V < 1 || K < 1 || K > V || chunk < 1) return KD_ERR_INVALID_ARG;
+  if (!(tau > 0.f) || !isfinite(tau)) return KD_ERR_INVALID_ARG;
+  if (!aligned(h, 16) || !aligned(W, 16) || !aligned(t_vals, 16) || !aligned(t_idx, 16) ||
+      !aligned(ws, 1024))
+    return KD_ERR_INVALID_ARG;
+  if (dtype != KD_DTYPE_BF16 && dtype != KD_DTYPE_F32) return KD_ERR_UNSUPPORTED;
+  if (d % 8 != 0 || K > KD_MAX_K || V >= (int64_t(1) << 31) - 256 ||
+      d >= (int64_t(1) << 31) || T >= (int64_t(1) << 40))
+    return KD_ERR_UNSUPPORTED;
+  if (ws_bytes < kd::ws_layout(T, d, V, K, chunk, dtype).total) return KD_ERR_WORKSPACE;
+  return KD_OK;
+}
+
+kd_status kd_fused_kl_fwd(const void* h, const void* W, int dtype, int64_t T, int64_t d,
+                          int64_t V, const float* t_vals, const int32_t* t_idx, int K,
+                          int64_t chunk, float temperature, float* loss, float* lse,
+                          float* kl_rows, void* ws, size_t ws_bytes, void* stream) {
+  kd_status st =
+      validate_loss(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, ws, ws_bytes);
+  if (st != KD_OK) return st;
+  if (!loss || !lse) return KD_ERR_INVALID_ARG;
+  if (!aligned(loss, 4) || !aligned(lse, 16) || (kl_rows && !aligned(kl_rows, 16)))
+    return KD_ERR_INVALID_ARG;
+  const int sms = num_sms_current();
+  if (sms <= 0) return KD_ERR_CUDA;
+  return kd::fused_fwd(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, loss, lse,
+                       kl_rows, ws, static_cast<cudaStream_t>(stream), sms, g_wait_limit_ns);
+}
+
+kd_status kd_fused_kl_bwd(const void* h, const void* W, int dtype, int64_t T, int64_t d,
+                          int64_t V, const float* t_vals, const int32_t* t_idx, int K,
+                          int64_t chunk, float temperature, const float* lse,
+                          const float* grad_loss, void* dH, float* dW, int accumulate_dW,
+                          void* ws, size_t ws_bytes, void* stream) {
+  kd_status st =
+      validate_loss(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, ws, ws_bytes);
+  if (st != KD_OK) return st;
+  if (!lse || !dH || !dW) return KD_ERR_INVALID_ARG;
+  if (!aligned(lse, 16) || !aligned(dH, 16) || !aligned(dW, 16) ||
+      (grad_loss && !aligned(grad_loss, 4)))
+    return KD_ERR_INVALID_ARG;
+  const int sms = num_sms_current();
+  if (sms <= 0) return KD_ERR_CUDA;
+  return kd::fused_bwd(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, lse,
+                       grad_loss, dH, dW, accumulate_dW, ws, static_cast<cudaStream_t>(stream),
+                       sms, g_wait_limit_ns);
+}
+
+kd_status kd_read_device_status(const void* ws, void* stream) {
+  if (!ws) return KD_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, s) != cudaSuccess) return KD_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KD_ERR_CUDA;
+  return static_cast<kd_status>(v);
+}
+
+uint64_t kd_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+kd_status kd_profile_attach(void* const* start_events, void* const* end_events, int* kinds,
+                            double* flops, int capacity, int kind_mask) {
+  if (!start_events || !end_events || capacity < 1) return KD_ERR_INVALID_ARG;
+  g_prof.start = start_events;
+  g_prof.end = end_events;
+  g_prof.kinds = kinds;
+  g_prof.flops = flops;
+  g_prof.capacity = capacity;
+  g_prof.mask = kind_mask;
+  g_prof.n = 0;
+  g_prof.armed = false;
+  return KD_OK;
+}
+
+int kd_profile_detach(void) {
+  const int n = g_prof.n;
+  g_prof = Profile{};
+  return n;
+}
+
+kd_status kd_set_wait_limit_ns(uint64_t limit_ns) {
+  if (limit_ns < 1000) return KD_ERR_INVALID_ARG;
+  g_wait_limit_ns = limit_ns;
+  return KD_OK;
+}
+
+kd_status kd_debug_wait_probe(void* ws, size_t ws_bytes, uint64_t limit_ns, void* stream) {
+  if (!ws || ws_bytes < 1024 || !aligned(ws, 1024)) return KD_ERR_INVALID_ARG;
+  if (limit_ns < 1000 || limit_ns > 10000000000ull) return KD_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return KD_ERR_CUDA;
+  if (kd::launch_wait_probe(static_cast<uint32_t*>(ws), limit_ns, s) != cudaSuccess)
+    return KD_ERR_CUDA;
+  return KD_OK;
+}
+
+}  // extern "C"

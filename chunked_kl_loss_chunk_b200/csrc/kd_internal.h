@@ -1,0 +1,40 @@
+// kd_internal.h -- declarations shared by the translation units of libkd.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "kd.h"
+
+namespace kd {
+
+// Byte offsets of the regions of a fused-loss workspace.
+struct WsLayout {
+  size_t p_sorted = 0, idx_sorted = 0, stats = 0, kl = 0, scratch = 0, total = 0;
+  int64_t ldz = 0;  // row pitch (elements) of the dz scratch
+};
+
+WsLayout ws_layout(int64_t T, int64_t d, int64_t V, int K, int64_t chunk, int dtype);
+
+kd_status fused_fwd(const void* h, const void* W, int dtype, int64_t T, int64_t d, int64_t V,
+                    const float* t_vals, const int32_t* t_idx, int K, int64_t chunk, float tau,
+                    float* loss, float* lse, float* kl_rows, void* ws, cudaStream_t s,
+                    int num_sms, uint64_t limit_ns);
+
+kd_status fused_bwd(const void* h, const void* W, int dtype, int64_t T, int64_t d, int64_t V,
+                    const float* t_vals, const int32_t* t_idx, int K, int64_t chunk, float tau,
+                    const float* lse, const float* grad_loss, void* dH, float* dW,
+                    int accumulate, void* ws, cudaStream_t s, int num_sms, uint64_t limit_ns);
+
+cudaError_t launch_topk_bf16(const void* logits, int64_t T, int64_t V, int K, float* out_vals,
+                             int32_t* out_idx, cudaStream_t stream, int num_sms);
+
+cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
+
+// Launch accounting and optional per-GEMM event recording.
+void count_launch();
+void profile_before(int kind, double flops, cudaStream_t s);
+void profile_after(cudaStream_t s);
+
+}  // namespace kd

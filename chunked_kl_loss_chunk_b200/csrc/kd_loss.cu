@@ -1,0 +1,463 @@
+// kd_loss.cu -- the fused chunked top-K KL loss: cache preparation, the chunk
+// loop of the forward (projection + logsumexp + gather fused into the GEMM
+// epilogue, then a per-row combine) and of the backward (projection recomputed
+// with dz formed in the epilogue, then dH = dz W and dW += dz^T h).
+//
+// Method: developersdigest.tech "Distilling an LLM on One GPU", section "The two
+// changes" (one chunk of positions at a time: project to logits for that chunk,
+// fold into the running loss, discard; the backward recomputes each chunk);
+// scitechpulse.com "New distillation trick ..." (the output projection is
+// folded into the loss so the student's logits grid is never materialised).
+#include <math.h>
+#include <string.h>
+
+#include "kd_gemm.cuh"
+#include "kd_internal.h"
+
+namespace kd {
+
+// ----------------------------------------------------------------------------
+// K2: cache prep.  One warp per position: p = softmax(vals / tau) over the K
+// cached logits, S = sum p, sum p log p, then the (index, p) pairs sorted by
+// index ascending.  Indices outside [0, V) or repeated in a row record
+// KD_ERR_BAD_INDEX; such entries get p = 0 and are moved past V.
+// ----------------------------------------------------------------------------
+constexpr int PREP_WARPS = 4;
+constexpr int PREP_MAXK = 1024;
+
+__global__ void __launch_bounds__(PREP_WARPS * 32)
+prep_kernel(const float* __restrict__ vals, const int32_t* __restrict__ idx, int64_t T, int K,
+            int64_t V, float inv_tau, int32_t* __restrict__ idx_sorted,
+            float* __restrict__ p_sorted, float2* __restrict__ stats, uint32_t* status) {
+  extern __shared__ __align__(16) unsigned char prep_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint64_t* buf = reinterpret_cast<uint64_t*>(prep_smem) + warp * PREP_MAXK;
+  int np = 1;
+  while (np < K) np <<= 1;
+
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * PREP_WARPS + warp; t < T;
+       t += static_cast<int64_t>(gridDim.x) * PREP_WARPS) {
+    const float* vr = vals + t * K;
+    const int32_t* ir = idx + t * K;
+    float mx = -INFINITY;
+    for (int k = lane; k < K; k += 32) mx = fmaxf(mx, vr[k] * inv_tau);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float se = 0.f;
+    for (int k = lane; k < K; k += 32) se += expf(vr[k] * inv_tau - mx);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
+    const float inv_se = 1.f / se;
+    float S = 0.f, plogp = 0.f;
+    bool bad = false;
+    for (int k = lane; k < K; k += 32) {
+      float p = expf(vr[k] * inv_tau - mx) * inv_se;
+      int32_t i = ir[k];
+      if (i < 0 || static_cast<int64_t>(i) >= V) {
+        bad = true;
+        p = 0.f;
+        i = INT32_MAX;
+      }
+      S += p;
+      if (p > 0.f) plogp += p * logf(p);
+      buf[k] = (static_cast<uint64_t>(static_cast<uint32_t>(i)) << 32) | __float_as_uint(p);
+    }
+    for (int k = K + lane; k < np; k += 32) buf[k] = ~0ull;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      S += __shfl_xor_sync(0xffffffffu, S, o);
+      plogp += __shfl_xor_sync(0xffffffffu, plogp, o);
+    }
+    __syncwarp();
+    // bitonic sort of np entries by index (upper 32 bits), ascending
+    for (int kk = 2; kk <= np; kk <<= 1) {
+      for (int j = kk >> 1; j > 0; j >>= 1) {
+        for (int i = lane; i < np; i += 32) {
+          const int ixj = i ^ j;
+          if (ixj > i) {
+            const uint64_t x = buf[i], y = buf[ixj];
+            const bool up = (i & kk) == 0;
+            if ((x > y) == up) {
+              buf[i] = y;
+              buf[ixj] = x;
+            }
+          }
+        }
+        __syncwarp();
+      }
+    }
+    for (int k = lane; k < K; k += 32) {
+      const uint64_t e = buf[k];
+      const uint32_t i = static_cast<uint32_t>(e >> 32);
+      if (k > 0 && i != 0x7FFFFFFFu && static_cast<uint32_t>(buf[k - 1] >> 32) == i) bad = true;
+      idx_sorted[t * K + k] = static_cast<int32_t>(i);
+      p_sorted[t * K + k] = __uint_as_float(static_cast<uint32_t>(e));
+    }
+    if (lane == 0) stats[t] = make_float2(S, plogp);
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(status, KD_ERR_BAD_INDEX);
+    __syncwarp();
+  }
+}
+
+// ----------------------------------------------------------------------------
+// K4: combine the per-(row, vocab tile) partials of one chunk.  One warp per
+// row; lane l merges tiles l, l+32, ... in order, then a fixed shuffle tree.
+//   LSE_t = M/tau + ln S,  KL_t = sum p log p - G/tau + (sum p) LSE_t
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void merge_lse(float& m, float& s, float m2, float s2, float zs) {
+  const float nm = fmaxf(m, m2);
+  if (nm == -INFINITY) return;
+  s = s * exp2f((m - nm) * zs) + s2 * exp2f((m2 - nm) * zs);
+  m = nm;
+}
+
+__global__ void __launch_bounds__(256)
+combine_kernel(const float4* __restrict__ partials, int rows, int n_tiles, int64_t row0,
+               float zscale, float inv_tau, const float2* __restrict__ stats,
+               float* __restrict__ lse, float* __restrict__ kl) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  const float4* pr = partials + static_cast<int64_t>(warp) * n_tiles;
+  float m = -INFINITY, s = 0.f, gsum = 0.f;
+  for (int j = lane; j < n_tiles; j += 32) {
+    const float4 q = pr[j];
+    merge_lse(m, s, q.x, q.y, zscale);
+    gsum += q.z;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    const float g2 = __shfl_xor_sync(0xffffffffu, gsum, o);
+    // xor partners combine symmetrically; use a canonical operand order so that
+    // both lanes compute bit-identical results.
+    if (lane & o) {
+      float mm = m2, ss = s2;
+      merge_lse(mm, ss, m, s, zscale);
+      m = mm;
+      s = ss;
+      gsum = g2 + gsum;
+    } else {
+      merge_lse(m, s, m2, s2, zscale);
+      gsum = gsum + g2;
+    }
+  }
+  if (lane == 0) {
+    const int64_t t = row0 + warp;
+    const float L = m * inv_tau + logf(s);
+    const float2 st = stats[t];
+    lse[t] = L;
+    kl[t] = st.y - gsum * inv_tau + st.x * L;
+  }
+}
+
+// Deterministic mean of kl[0..T): one block, fixed per-thread strides, fixed
+// tree; fp64 accumulation.
+__global__ void __launch_bounds__(1024)
+mean_kernel(const float* __restrict__ kl, int64_t T, float* __restrict__ loss) {
+  __shared__ double part[1024];
+  double acc = 0.0;
+  for (int64_t i = threadIdx.x; i < T; i += 1024) acc += static_cast<double>(kl[i]);
+  part[threadIdx.x] = acc;
+  __syncthreads();
+  for (int s = 512; s > 0; s >>= 1) {
+    if (threadIdx.x < s) part[threadIdx.x] += part[threadIdx.x + s];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) *loss = static_cast<float>(part[0] / static_cast<double>(T));
+}
+
+// Failure-detection probe: waits on a barrier that nothing arrives at.
+__global__ void wait_probe_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, limit_ns, status);
+}
+
+// ----------------------------------------------------------------------------
+// Host side.
+// ----------------------------------------------------------------------------
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D row-major tensor [outer, inner] with the given row pitch (elements),
+// 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* map, const void* base, bool f32, uint64_t inner, uint64_t outer,
+              uint64_t pitch_elems, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const uint64_t es = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch_elems * es};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                  2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename Elem, int A_MN, int B_MN, int EPI>
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmArgs g,
+                        cudaStream_t s, int num_sms) {
+  static constexpr int kKind[4] = {KD_GEMM_FWD_LSE, KD_GEMM_BWD_DZ, KD_GEMM_DH, KD_GEMM_DW};
+  auto kern = gemm_kernel<Elem, A_MN, B_MN, EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       GEMM_SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int tiles = g.m_tiles * g.n_tiles;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  profile_before(kKind[EPI], 2.0 * g.M * static_cast<double>(g.N) * g.K, s);
+  kern<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, s>>>(ta, tb, g);
+  count_launch();
+  profile_after(s);
+  return cudaGetLastError();
+}
+
+inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
+
+}  // namespace
+
+WsLayout ws_layout(int64_t T, int64_t d, int64_t V, int K, int64_t chunk, int dtype) {
+  (void)d;
+  WsLayout L;
+  const size_t es = dtype == KD_DTYPE_F32 ? 4 : 2;
+  auto al = [](size_t x) { return (x + 1023) & ~static_cast<size_t>(1023); };
+  size_t off = 1024;  // status word + reserved
+  L.p_sorted = off;
+  off = al(off + static_cast<size_t>(T) * K * 4);
+  L.idx_sorted = off;
+  off = al(off + static_cast<size_t>(T) * K * 4);
+  L.stats = off;
+  off = al(off + static_cast<size_t>(T) * 8);
+  L.kl = off;
+  off = al(off + static_cast<size_t>(T) * 4);
+  const int64_t rows = chunk < T ? chunk : T;
+  L.ldz = ((V + 63) / 64) * 64;
+  const size_t n_tiles = static_cast<size_t>((V + BN - 1) / BN);
+  const size_t part = static_cast<size_t>(rows) * n_tiles * 16;
+  const size_t dz = static_cast<size_t>(rows) * static_cast<size_t>(L.ldz) * es;
+  L.scratch = off;
+  off = al(off + (part > dz ? part : dz));
+  L.total = off;
+  return L;
+}
+
+template <typename Elem>
+static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t d, int64_t V,
+                          const float* t_vals, const int32_t* t_idx, int K, int64_t chunk,
+                          float tau, float* loss, float* lse, float* kl_rows, void* ws,
+                          cudaStream_t s, int num_sms, uint64_t limit_ns) {
+  constexpr bool F32 = sizeof(Elem) == 4;
+  constexpr int BK = ElemCfg<Elem>::BK;
+  const WsLayout L = ws_layout(T, d, V, K, chunk, F32 ? KD_DTYPE_F32 : KD_DTYPE_BF16);
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(w);
+  int32_t* idx_s = reinterpret_cast<int32_t*>(w + L.idx_sorted);
+  float* p_s = reinterpret_cast<float*>(w + L.p_sorted);
+  float2* stats = reinterpret_cast<float2*>(w + L.stats);
+  float* kl = kl_rows ? kl_rows : reinterpret_cast<float*>(w + L.kl);
+  float4* part = reinterpret_cast<float4*>(w + L.scratch);
+
+  if (cudaMemsetAsync(status, 0, 4, s) != cudaSuccess) return KD_ERR_CUDA;
+  const float inv_tau = 1.f / tau;
+  {
+    const int64_t blocks64 = (T + PREP_WARPS - 1) / PREP_WARPS;
+    const int blocks = static_cast<int>(blocks64 < 65535 * 16 ? blocks64 : 65535 * 16);
+    prep_kernel<<<blocks, PREP_WARPS * 32, PREP_WARPS * PREP_MAXK * 8, s>>>(
+        t_vals, t_idx, T, K, V, inv_tau, idx_s, p_s, stats, status);
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+  }
+  CUtensorMap tW;
+  if (!make_map(&tW, W, F32, d, V, d, BK, BN)) return KD_ERR_CUDA;
+  const float zscale = 1.4426950408889634f * inv_tau;
+  for (int64_t c0 = 0; c0 < T; c0 += chunk) {
+    const int64_t rows = (T - c0) < chunk ? (T - c0) : chunk;
+    CUtensorMap tH;
+    const Elem* hc = static_cast<const Elem*>(h) + c0 * d;
+    if (!make_map(&tH, hc, F32, d, rows, d, BK, BM)) return KD_ERR_CUDA;
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    g.M = static_cast<int32_t>(rows);
+    g.N = static_cast<int32_t>(V);
+    g.K = static_cast<int32_t>(d);
+    g.m_tiles = cdiv(rows, BM);
+    g.n_tiles = cdiv(V, BN);
+    g.k_blocks = cdiv(d, BK);
+    g.m_fastest = 1;
+    g.row0 = c0;
+    g.V = V;
+    g.Ktop = K;
+    g.zscale = zscale;
+    g.idx_sorted = idx_s;
+    g.p_sorted = p_s;
+    g.row_stats = stats;
+    g.partials = part;
+    g.status = status;
+    g.wait_limit_ns = limit_ns;
+    if (launch_gemm<Elem, 0, 0, EPI_FWD_LSE>(tH, tW, g, s, num_sms) != cudaSuccess)
+      return KD_ERR_CUDA;
+    const int cblocks = cdiv(rows * 32, 256);
+    combine_kernel<<<cblocks, 256, 0, s>>>(part, static_cast<int>(rows), g.n_tiles, c0, zscale,
+                                           inv_tau, stats, lse, kl);
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+  }
+  mean_kernel<<<1, 1024, 0, s>>>(kl, T, loss);
+  count_launch();
+  if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+  return KD_OK;
+}
+
+template <typename Elem>
+static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, int64_t V,
+                          const float* t_vals, const int32_t* t_idx, int K, int64_t chunk,
+                          float tau, const float* lse, const float* grad_loss, void* dH,
+                          float* dW, int accumulate, void* ws, cudaStream_t s, int num_sms,
+                          uint64_t limit_ns) {
+  constexpr bool F32 = sizeof(Elem) == 4;
+  constexpr int BK = ElemCfg<Elem>::BK;
+  constexpr int INNER = ROW_BYTES / sizeof(Elem);
+  const WsLayout L = ws_layout(T, d, V, K, chunk, F32 ? KD_DTYPE_F32 : KD_DTYPE_BF16);
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(w);
+  int32_t* idx_s = reinterpret_cast<int32_t*>(w + L.idx_sorted);
+  float* p_s = reinterpret_cast<float*>(w + L.p_sorted);
+  float2* stats = reinterpret_cast<float2*>(w + L.stats);
+  Elem* dz = reinterpret_cast<Elem*>(w + L.scratch);
+
+  if (cudaMemsetAsync(status, 0, 4, s) != cudaSuccess) return KD_ERR_CUDA;
+  const float inv_tau = 1.f / tau;
+  {
+    const int64_t blocks64 = (T + PREP_WARPS - 1) / PREP_WARPS;
+    const int blocks = static_cast<int>(blocks64 < 65535 * 16 ? blocks64 : 65535 * 16);
+    prep_kernel<<<blocks, PREP_WARPS * 32, PREP_WARPS * PREP_MAXK * 8, s>>>(
+        t_vals, t_idx, T, K, V, inv_tau, idx_s, p_s, stats, status);
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+  }
+  CUtensorMap tW_k, tW_mn;
+  if (!make_map(&tW_k, W, F32, d, V, d, BK, BN)) return KD_ERR_CUDA;      // [V, d], K = d
+  if (!make_map(&tW_mn, W, F32, d, V, d, INNER, BK)) return KD_ERR_CUDA;  // K = V rows, N = d
+  const float zscale = 1.4426950408889634f * inv_tau;
+  const float inv_T_tau = static_cast<float>(1.0 / (static_cast<double>(T) * tau));
+  for (int64_t c0 = 0; c0 < T; c0 += chunk) {
+    const int64_t rows = (T - c0) < chunk ? (T - c0) : chunk;
+    const Elem* hc = static_cast<const Elem*>(h) + c0 * d;
+    CUtensorMap tH_k, tH_mn, tDz_k, tDz_mn;
+    if (!make_map(&tH_k, hc, F32, d, rows, d, BK, BM)) return KD_ERR_CUDA;
+    if (!make_map(&tH_mn, hc, F32, d, rows, d, INNER, BK)) return KD_ERR_CUDA;
+    if (!make_map(&tDz_k, dz, F32, V, rows, L.ldz, BK, BM)) return KD_ERR_CUDA;
+    if (!make_map(&tDz_mn, dz, F32, V, rows, L.ldz, INNER, BK)) return KD_ERR_CUDA;
+
+    // (1) recompute z = h_c W^T; epilogue writes dz_c [rows, ldz]
+    GemmArgs g;
+    memset(&g, 0, sizeof(g));
+    g.M = static_cast<int32_t>(rows);
+    g.N = static_cast<int32_t>(V);
+    g.K = static_cast<int32_t>(d);
+    g.m_tiles = cdiv(rows, BM);
+    g.n_tiles = cdiv(V, BN);
+    g.k_blocks = cdiv(d, BK);
+    g.m_fastest = 1;
+    g.row0 = c0;
+    g.V = V;
+    g.Ktop = K;
+    g.zscale = zscale;
+    g.idx_sorted = idx_s;
+    g.p_sorted = p_s;
+    g.row_stats = stats;
+    g.lse = lse;
+    g.grad_loss = grad_loss;
+    g.inv_T_tau = inv_T_tau;
+    g.out = dz;
+    g.ldo = L.ldz;
+    g.status = status;
+    g.wait_limit_ns = limit_ns;
+    if (launch_gemm<Elem, 0, 0, EPI_BWD_DZ>(tH_k, tW_k, g, s, num_sms) != cudaSuccess)
+      return KD_ERR_CUDA;
+
+    // (2) dH_c = dz_c W : M = rows, N = d, K = V; A K-major, B MN-major
+    GemmArgs gh = g;
+    gh.N = static_cast<int32_t>(d);
+    gh.K = static_cast<int32_t>(V);
+    gh.n_tiles = cdiv(d, BN);
+    gh.k_blocks = cdiv(V, BK);
+    gh.m_fastest = 1;
+    gh.out = dH;
+    gh.ldo = d;
+    if (launch_gemm<Elem, 0, 1, EPI_STORE_H>(tDz_k, tW_mn, gh, s, num_sms) != cudaSuccess)
+      return KD_ERR_CUDA;
+
+    // (3) dW (+)= dz_c^T h_c : M = V, N = d, K = rows; both operands MN-major
+    GemmArgs gw = g;
+    gw.M = static_cast<int32_t>(V);
+    gw.N = static_cast<int32_t>(d);
+    gw.K = static_cast<int32_t>(rows);
+    gw.m_tiles = cdiv(V, BM);
+    gw.n_tiles = cdiv(d, BN);
+    gw.k_blocks = cdiv(rows, BK);
+    gw.m_fastest = 0;              // tiles sharing one dz slab run together
+    gw.row0 = 0;
+    gw.out = dW;
+    gw.ldo = d;
+    gw.accumulate = (accumulate || c0 > 0) ? 1 : 0;
+    if (launch_gemm<Elem, 1, 1, EPI_ACCUM_W>(tDz_mn, tH_mn, gw, s, num_sms) != cudaSuccess)
+      return KD_ERR_CUDA;
+  }
+  return KD_OK;
+}
+
+kd_status fused_fwd(const void* h, const void* W, int dtype, int64_t T, int64_t d, int64_t V,
+                    const float* t_vals, const int32_t* t_idx, int K, int64_t chunk, float tau,
+                    float* loss, float* lse, float* kl_rows, void* ws, cudaStream_t s,
+                    int num_sms, uint64_t limit_ns) {
+  if (dtype == KD_DTYPE_F32)
+    return fwd_impl<float>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, loss, lse, kl_rows, ws,
+                           s, num_sms, limit_ns);
+  return fwd_impl<__nv_bfloat16>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, loss, lse,
+                                 kl_rows, ws, s, num_sms, limit_ns);
+}
+
+kd_status fused_bwd(const void* h, const void* W, int dtype, int64_t T, int64_t d, int64_t V,
+                    const float* t_vals, const int32_t* t_idx, int K, int64_t chunk, float tau,
+                    const float* lse, const float* grad_loss, void* dH, float* dW,
+                    int accumulate, void* ws, cudaStream_t s, int num_sms, uint64_t limit_ns) {
+  if (dtype == KD_DTYPE_F32)
+    return bwd_impl<float>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, lse, grad_loss, dH, dW,
+                           accumulate, ws, s, num_sms, limit_ns);
+  return bwd_impl<__nv_bfloat16>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, lse, grad_loss,
+                                 dH, dW, accumulate, ws, s, num_sms, limit_ns);
+}
+
+cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t s) {
+  wait_probe_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace kd

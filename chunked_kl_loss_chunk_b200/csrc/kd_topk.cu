@@ -1,0 +1,367 @@
+// kd_topk.cu -- top-K cache build (the offline teacher cache of the
+// developersdigest.tech page "Distilling an LLM on One GPU", section "The two
+// changes": the teacher's top-100 tokens per position are computed once).
+//
+// Per row of bf16 teacher logits, select the K entries ranked by
+// (value descending, index ascending), +0 == -0, NaN below -inf.
+//
+// Design (HBM-bound streaming select):
+//   1. sample: 4096-bin histogram (order key >> 4) of the first min(V, 4096)
+//      elements gives a threshold bin L whose count from the top covers about
+//      4K expected row elements.  L is turned into a float threshold tf with
+//      key(x) >= L<<4  <=>  x >= tf  for every non-NaN x.
+//   2. stream: one coalesced 16-byte-vector pass over the row; each element is
+//      one float compare against tf; the rare survivors are appended to a
+//      shared-memory candidate buffer.
+//   3. if K <= survivors <= capacity, the top K of the row are exactly the top
+//      K of the survivors: bitonic-sort them by the composite (key desc,
+//      index asc) and write the first K.
+//   4. otherwise (ties, NaN-heavy or adversarially ordered rows) an exact
+//      3-pass histogram select runs instead (passes 2-3 hit L2).
+#include "kd_common.cuh"
+#include "kd_internal.h"
+
+namespace kd {
+
+constexpr int TK_THREADS = 512;
+constexpr int TK_BINS = 4096;       // bins of (order key >> 4)
+constexpr int TK_SAMPLE = 4096;
+constexpr int TK_CAND_CAP = 2048;
+constexpr int TK_SEL_CAP = 1024;    // >= K
+
+// Order-preserving 16-bit key of a bf16 bit pattern: NaN -> 0 (lowest),
+// -0 -> key of +0, otherwise a monotone map of the value.
+__device__ __forceinline__ uint32_t bf16_order_key(uint32_t b) {
+  b &= 0xFFFFu;
+  const uint32_t mag = b & 0x7FFFu;
+  if (mag > 0x7F80u) return 0u;
+  if (mag == 0u) return 0x8000u;
+  return (b & 0x8000u) ? (~b & 0xFFFFu) : (b | 0x8000u);
+}
+
+// Ascending order of this 64-bit composite = key descending, index ascending.
+__device__ __forceinline__ uint64_t composite(uint32_t key, uint32_t idx) {
+  return (static_cast<uint64_t>(0xFFFFu - key) << 32) | idx;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
+  return __uint_as_float((b & 0xFFFFu) << 16);
+}
+
+struct TopkSmem {
+  uint32_t hist[TK_BINS];
+  uint64_t cand[TK_CAND_CAP];
+  uint64_t sel[TK_SEL_CAP];
+  uint32_t warp_tot[TK_THREADS / 32 + 1];
+  uint32_t hist16[16];
+  uint32_t n_cand;
+  uint32_t n_sel;
+  uint32_t thr_bin;
+  uint32_t thr_above;
+  uint32_t eq_base;
+};
+
+// Exclusive block scan of one value per thread (TK_THREADS threads); also
+// returns the block total.  warp_tot needs TK_THREADS/32 + 1 entries.
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_tot,
+                                                    uint32_t& total) {
+  constexpr int NW = TK_THREADS / 32;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[w] = x;
+  __syncthreads();
+  if (w == 0) {
+    const uint32_t t = lane < NW ? warp_tot[lane] : 0u;
+    uint32_t s = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane < NW) warp_tot[lane] = s - t;
+    if (lane == NW - 1) warp_tot[NW] = s;
+  }
+  __syncthreads();
+  const uint32_t r = warp_tot[w] + x - v;
+  total = warp_tot[NW];
+  __syncthreads();
+  return r;
+}
+
+// Highest bin b with (count of bins > b) < target <= (count of bins >= b).
+// If the histogram holds fewer than `target` elements, returns bin 0.
+// Writes sm.thr_bin / sm.thr_above.
+__device__ void find_threshold_bin(TopkSmem& sm, uint32_t target) {
+  constexpr int PER = TK_BINS / TK_THREADS;  // 8
+  const int t = threadIdx.x;
+  const int hi = TK_BINS - PER * t;          // thread 0 owns the top bins
+  uint32_t local = 0;
+#pragma unroll
+  for (int j = 1; j <= PER; ++j) local += sm.hist[hi - j];
+  uint32_t total;
+  uint32_t above = block_excl_scan(local, sm.warp_tot, total);
+  if (t == 0 && total < target) {
+    sm.thr_bin = 0;
+    sm.thr_above = 0;
+  }
+  if (above < target && above + local >= target) {
+#pragma unroll 1
+    for (int j = 1; j <= PER; ++j) {
+      const uint32_t c = sm.hist[hi - j];
+      if (above + c >= target) {
+        sm.thr_bin = hi - j;
+        sm.thr_above = above;
+        break;
+      }
+      above += c;
+    }
+  }
+  __syncthreads();
+}
+
+// In-place ascending bitonic sort of n (power of two, <= cap) entries.
+__device__ void bitonic_sort(uint64_t* a, int n) {
+  for (int k = 2; k <= n; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < n; i += TK_THREADS) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const uint64_t x = a[i], y = a[ixj];
+          const bool up = (i & k) == 0;
+          if ((x > y) == up) {
+            a[i] = y;
+            a[ixj] = x;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+__device__ __forceinline__ int next_pow2(int n) {
+  int p = 1;
+  while (p < n) p <<= 1;
+  return p;
+}
+
+// Visit every element of a row with 16-byte vector loads where possible.
+template <class F>
+__device__ __forceinline__ void for_each_elem(const uint16_t* __restrict__ row, int64_t V, F&& f) {
+  const uintptr_t addr = reinterpret_cast<uintptr_t>(row);
+  int64_t head = ((16 - (addr & 15)) & 15) >> 1;
+  if (head > V) head = V;
+  for (int64_t i = threadIdx.x; i < head; i += TK_THREADS) f(row[i], static_cast<uint32_t>(i));
+  const int64_t nvec = (V - head) >> 3;
+  const uint4* vp = reinterpret_cast<const uint4*>(row + head);
+  for (int64_t j = threadIdx.x; j < nvec; j += TK_THREADS) {
+    const uint4 q = __ldcs(vp + j);
+    const uint32_t base = static_cast<uint32_t>(head + (j << 3));
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      f(w[u] & 0xFFFFu, base + 2 * u);
+      f(w[u] >> 16, base + 2 * u + 1);
+    }
+  }
+  for (int64_t i = head + (nvec << 3) + threadIdx.x; i < V; i += TK_THREADS)
+    f(row[i], static_cast<uint32_t>(i));
+}
+
+__global__ void __launch_bounds__(TK_THREADS)
+topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int K,
+                 float* __restrict__ out_vals, int32_t* __restrict__ out_idx) {
+  extern __shared__ __align__(16) unsigned char tk_smem_raw[];
+  TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_smem_raw);
+  const int tid = threadIdx.x;
+
+  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+    const uint16_t* row = logits + t * V;
+
+    // ---- 1. sample threshold -------------------------------------------------
+    for (int b = tid; b < TK_BINS; b += TK_THREADS) sm.hist[b] = 0u;
+    if (tid == 0) {
+      sm.n_cand = 0;
+      sm.n_sel = 0;
+    }
+    __syncthreads();
+    const int64_t S = V < TK_SAMPLE ? V : TK_SAMPLE;
+    for (int64_t i = tid; i < S; i += TK_THREADS)
+      atomicAdd(&sm.hist[bf16_order_key(row[i]) >> 4], 1u);
+    __syncthreads();
+    uint32_t target;
+    if (S == V) {
+      target = static_cast<uint32_t>(K);
+    } else {
+      const double want = 4.0 * K * static_cast<double>(S) / static_cast<double>(V);
+      target = static_cast<uint32_t>(ceil(want));
+      if (target < 1u) target = 1u;
+    }
+    find_threshold_bin(sm, target);
+    const uint32_t L = sm.thr_bin << 4;   // candidate iff order key >= L
+    // Float threshold equivalent on non-NaN values: key >= L <=> x >= tf.
+    float tf = 0.f;
+    bool take_all = false;
+    if (L == 0u) {
+      take_all = true;                              // threshold inside the NaN bin
+    } else if (L <= 0x7Fu) {
+      tf = -INFINITY;                               // every non-NaN value qualifies
+    } else if (L < 0x8000u) {
+      tf = bf16_bits_to_float((~L) & 0xFFFFu);      // the negative value with key L
+    } else {
+      tf = bf16_bits_to_float(L & 0x7FFFu);         // +0 when L == 0x8000
+    }
+
+    // ---- 2. stream the row, keep survivors ------------------------------------
+    for_each_elem(row, V, [&](uint32_t bits, uint32_t i) {
+      const float x = bf16_bits_to_float(bits);
+      if (take_all || x >= tf) {
+        const uint32_t pos = atomicAdd(&sm.n_cand, 1u);
+        if (pos < TK_CAND_CAP) sm.cand[pos] = composite(bf16_order_key(bits), i);
+      }
+    });
+    __syncthreads();
+    const uint32_t n = sm.n_cand;
+
+    if (n >= static_cast<uint32_t>(K) && n <= static_cast<uint32_t>(TK_CAND_CAP)) {
+      // ---- 3. exact select among survivors -------------------------------------
+      const int np = next_pow2(static_cast<int>(n));
+      for (int i = static_cast<int>(n) + tid; i < np; i += TK_THREADS) sm.cand[i] = ~0ull;
+      __syncthreads();
+      bitonic_sort(sm.cand, np);
+      for (int k = tid; k < K; k += TK_THREADS) {
+        const uint64_t c = sm.cand[k];
+        const uint32_t i = static_cast<uint32_t>(c);
+        out_idx[t * K + k] = static_cast<int32_t>(i);
+        out_vals[t * K + k] = bf16_bits_to_float(row[i]);
+      }
+      __syncthreads();
+      continue;
+    }
+
+    // ---- 4. exact 3-pass fallback --------------------------------------------
+    // Pass A: full-row histogram of key >> 4.
+    for (int b = tid; b < TK_BINS; b += TK_THREADS) sm.hist[b] = 0u;
+    if (tid < 16) sm.hist16[tid] = 0u;
+    if (tid == 0) {
+      sm.n_sel = 0;
+      sm.eq_base = 0;
+    }
+    __syncthreads();
+    for_each_elem(row, V, [&](uint32_t bits, uint32_t) {
+      atomicAdd(&sm.hist[bf16_order_key(bits) >> 4], 1u);
+    });
+    __syncthreads();
+    find_threshold_bin(sm, static_cast<uint32_t>(K));
+    const uint32_t b1 = sm.thr_bin, above1 = sm.thr_above;
+    if (tid == 0) sm.n_sel = 0;
+    __syncthreads();
+    // Pass B: keep bins above b1; histogram the low nibble inside b1.
+    for_each_elem(row, V, [&](uint32_t bits, uint32_t i) {
+      const uint32_t key = bf16_order_key(bits);
+      const uint32_t b = key >> 4;
+      if (b > b1) {
+        const uint32_t pos = atomicAdd(&sm.n_sel, 1u);
+        sm.sel[pos] = composite(key, i);
+      } else if (b == b1) {
+        atomicAdd(&sm.hist16[key & 15u], 1u);
+      }
+    });
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t above = above1;
+      uint32_t nib = 0;
+      for (int j = 15; j >= 0; --j) {
+        if (above + sm.hist16[j] >= static_cast<uint32_t>(K)) {
+          nib = static_cast<uint32_t>(j);
+          break;
+        }
+        above += sm.hist16[j];
+      }
+      sm.thr_bin = (b1 << 4) | nib;   // exact threshold key
+      sm.thr_above = above;           // number of keys strictly above it
+    }
+    __syncthreads();
+    const uint32_t Tk = sm.thr_bin;
+    const uint32_t need = static_cast<uint32_t>(K) - sm.thr_above;
+    // Pass C: keys in (Tk, bin b1 top] appended; keys == Tk taken in index order.
+    for (int64_t base = 0; base < V; base += 8 * TK_THREADS) {
+      const int64_t i0 = base + 8 * tid;
+      uint32_t eq_mask = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int64_t i = i0 + u;
+        if (i < V) {
+          const uint32_t key = bf16_order_key(row[i]);
+          if ((key >> 4) == b1 && key > Tk) {
+            const uint32_t pos = atomicAdd(&sm.n_sel, 1u);
+            sm.sel[pos] = composite(key, static_cast<uint32_t>(i));
+          } else if (key == Tk) {
+            eq_mask |= 1u << u;
+          }
+        }
+      }
+      uint32_t tile_total;
+      const uint32_t rank = block_excl_scan(__popc(eq_mask), sm.warp_tot, tile_total);
+      const uint32_t eb = sm.eq_base;
+      uint32_t r = eb + rank;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (eq_mask & (1u << u)) {
+          if (r < need) {
+            const uint32_t pos = atomicAdd(&sm.n_sel, 1u);
+            sm.sel[pos] = composite(Tk, static_cast<uint32_t>(i0 + u));
+          }
+          ++r;
+        }
+      }
+      __syncthreads();
+      if (tid == 0) sm.eq_base = eb + tile_total;
+      __syncthreads();
+    }
+    const int np = next_pow2(K);
+    for (int i = K + tid; i < np; i += TK_THREADS) sm.sel[i] = ~0ull;
+    __syncthreads();
+    bitonic_sort(sm.sel, np);
+    for (int k = tid; k < K; k += TK_THREADS) {
+      const uint64_t c = sm.sel[k];
+      const uint32_t i = static_cast<uint32_t>(c);
+      out_idx[t * K + k] = static_cast<int32_t>(i);
+      out_vals[t * K + k] = bf16_bits_to_float(row[i]);
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace kd
+
+// ----------------------------------------------------------------------------
+// Host launcher (called from kd_api.cu after argument validation).
+// ----------------------------------------------------------------------------
+namespace kd {
+
+cudaError_t launch_topk_bf16(const void* logits, int64_t T, int64_t V, int K, float* out_vals,
+                             int32_t* out_idx, cudaStream_t stream, int num_sms) {
+  const size_t smem = sizeof(TopkSmem);
+  cudaError_t e = cudaFuncSetAttribute(topk_bf16_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_bf16_kernel, TK_THREADS, smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) per_sm = 1;
+  int64_t grid = static_cast<int64_t>(num_sms) * per_sm;
+  if (grid > T) grid = T;
+  topk_bf16_kernel<<<static_cast<unsigned>(grid), TK_THREADS, smem, stream>>>(
+      static_cast<const uint16_t*>(logits), T, V, K, out_vals, out_idx);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace kd

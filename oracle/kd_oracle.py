@@ -63,7 +63,7 @@ def _as_f64(x) -> np.ndarray:
     x = np.asarray(x)
     if x.dtype == np.uint16 or x.dtype == np.int16:
         return bf16_bits_to_f64(x)
-    return x.astype(np.float64)
+    return x.astype(np.float64, copy=False)
 
 
 # ---------------------------------------------------------------------------

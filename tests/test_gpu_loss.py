@@ -1,0 +1,213 @@
+"""GPU parity of the fused chunked KL loss (forward and backward) against the
+fp64 oracle, through the C ABI.
+
+Tolerances (spec bar, written here):
+  * loss: relative error <= 1e-3;
+  * dH, dW: max|gpu - oracle| / max|oracle| <= 2e-2;
+  * lse: absolute error <= 1e-3 (bf16 operands multiply exactly and accumulate
+    in fp32, so z is good to ~1e-6 relative); <= 5e-3 for fp32 operands, which
+    the tensor cores read as tf32 (10-bit mantissa, ~5e-4 relative per operand).
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from chunked_kl_loss_chunk_b200 import inputs, kd
+from gpu_util import rel_maxabs, require_gpu, to_np_exact
+
+pytestmark = pytest.mark.gpu
+
+LOSS_RTOL = 1e-3
+GRAD_TOL = 2e-2
+
+
+def _run(T, d, V, K, chunk, dtype, tau=1.0, g=None, seed=0, acc_init=None):
+    h, W, vals, idx = inputs.make_loss_inputs(T, d, V, K, dtype=dtype, seed=seed, device="cuda")
+    loss, lse, kl, ws = kd.fused_kl_fwd(h, W, vals, idx, chunk, tau, kl_rows=True)
+    gl = None if g is None else torch.tensor(g, dtype=torch.float32, device="cuda")
+    dW0 = None
+    if acc_init is not None:
+        dW0 = torch.full((V, d), acc_init, dtype=torch.float32, device="cuda")
+    dH, dW, _ = kd.fused_kl_bwd(h, W, vals, idx, lse, chunk, tau, grad_loss=gl, ws=ws, dW=dW0,
+                                accumulate_dW=acc_init is not None)
+    torch.cuda.synchronize()
+    assert kd.read_device_status(ws) == kd.KD_OK
+    return dict(h=h, W=W, vals=vals, idx=idx, loss=loss, lse=lse, kl=kl, dH=dH, dW=dW)
+
+
+def _full_parity(r, tau=1.0, g=1.0, lse_tol=1e-3, acc_init=None):
+    h, W = to_np_exact(r["h"]), to_np_exact(r["W"])
+    vals, idx = r["vals"].cpu().numpy(), r["idx"].cpu().numpy()
+    loss, lse, kl = oracle.forward(h, W, vals, idx, tau)
+    dH, dW = oracle.backward(h, W, vals, idx, tau, g)
+    if acc_init is not None:
+        dW = dW + acc_init
+    gl = float(r["loss"].item())
+    assert abs(gl - loss) <= LOSS_RTOL * abs(loss), (gl, loss)
+    assert np.abs(r["lse"].cpu().numpy() - lse).max() <= lse_tol
+    assert np.abs(r["kl"].cpu().numpy() - kl).max() <= 10 * lse_tol
+    assert rel_maxabs(r["dH"].float().cpu().numpy(), dH) <= GRAD_TOL
+    assert rel_maxabs(r["dW"].cpu().numpy(), dW) <= GRAD_TOL
+    return dict(loss=loss, lse=lse, dH=dH, dW=dW)
+
+
+def test_tiny_fp32_config():
+    """T=256, d=256, V=4096, K=16, chunk=64, fp32 (the correctness config)."""
+    require_gpu()
+    r = _run(256, 256, 4096, 16, 64, torch.float32)
+    _full_parity(r, lse_tol=5e-3)
+
+
+@pytest.mark.parametrize("T,d,V,K,chunk,dtype", [
+    (300, 200, 5000, 16, 100, torch.bfloat16),     # ragged T, chunk, d (not /64), V (not /32)
+    (77, 72, 1003, 7, 33, torch.float32),          # odd V, tiny chunk
+    (129, 64, 257, 1, 129, torch.bfloat16),        # K = 1, V just over one tile
+    (64, 64, 64, 64, 16, torch.bfloat16),          # K = V
+    (520, 264, 2304, 100, 512, torch.bfloat16),    # several M and N tiles, K = 100
+])
+def test_ragged_shapes(T, d, V, K, chunk, dtype):
+    require_gpu()
+    r = _run(T, d, V, K, chunk, dtype, seed=T)
+    _full_parity(r, lse_tol=5e-3 if dtype == torch.float32 else 1e-3)
+
+
+def test_temperature_grad_scale_and_accumulate():
+    require_gpu()
+    r = _run(200, 128, 3000, 20, 64, torch.bfloat16, tau=2.0, g=3.0, acc_init=0.25)
+    _full_parity(r, tau=2.0, g=3.0, acc_init=0.25)
+
+
+def test_chunk_invariance_bitwise():
+    """Per-row results do not depend on the chunk size; the loss is bit-identical."""
+    require_gpu()
+    h, W, vals, idx = inputs.make_loss_inputs(384, 128, 6000, 16, dtype=torch.bfloat16, seed=3,
+                                              device="cuda")
+    outs = [kd.fused_kl_fwd(h, W, vals, idx, c, 1.0) for c in (384, 128, 100, 7)]
+    torch.cuda.synchronize()
+    for loss, lse, _, _ in outs[1:]:
+        assert torch.equal(loss, outs[0][0])
+        assert torch.equal(lse, outs[0][1])
+    dHs = [kd.fused_kl_bwd(h, W, vals, idx, outs[0][1], c, 1.0)[:2] for c in (384, 100)]
+    torch.cuda.synchronize()
+    assert torch.equal(dHs[0][0], dHs[1][0])                       # dH rows independent
+    assert rel_maxabs(dHs[1][1].cpu().numpy(), dHs[0][1].cpu().numpy()) <= 1e-5
+
+
+def test_zero_loss_when_student_reproduces_teacher():
+    """d = V = 64, W = I, h = teacher logits (bf16-exact) at idx and -60 elsewhere:
+    exact KL ~ 1e-24; fp32 cancellation of O(5) terms leaves ~1e-6."""
+    require_gpu()
+    T, V, K = 256, 64, 8
+    _, _, vals, idx = inputs.make_loss_inputs(T, V, V, K, dtype=torch.bfloat16, seed=5, device="cuda")
+    vals = vals.to(torch.bfloat16).float()
+    W = torch.eye(V, dtype=torch.bfloat16, device="cuda")
+    h = torch.full((T, V), -60.0, dtype=torch.float32, device="cuda")
+    h.scatter_(1, idx.long(), vals)
+    h = h.to(torch.bfloat16)
+    loss, lse, kl, _ = kd.fused_kl_fwd(h, W, vals.contiguous(), idx, 64, 1.0, kl_rows=True)
+    torch.cuda.synchronize()
+    assert abs(loss.item()) < 1e-5
+    assert kl.abs().max().item() < 1e-4
+
+
+def test_bad_index_recorded_not_faulted():
+    require_gpu()
+    h, W, vals, idx = inputs.make_loss_inputs(64, 64, 500, 8, dtype=torch.bfloat16, seed=1, device="cuda")
+    idx = idx.clone()
+    idx[3, 2] = 500 + 7          # out of range
+    idx[9, 1] = idx[9, 4]        # duplicate
+    loss, lse, _, ws = kd.fused_kl_fwd(h, W, vals, idx, 32, 1.0)
+    assert kd.read_device_status(ws) == kd.KD_ERR_BAD_INDEX
+    kd.fused_kl_bwd(h, W, vals, idx, lse, 32, 1.0, ws=ws)
+    assert kd.read_device_status(ws) == kd.KD_ERR_BAD_INDEX
+    # status is cleared by the next call on clean inputs
+    idx[3, 2] = 0 if int(idx[3].min()) != 0 else 499
+    _, _, vals2, idx2 = inputs.make_loss_inputs(64, 64, 500, 8, dtype=torch.bfloat16, seed=1, device="cuda")
+    kd.fused_kl_fwd(h, W, vals2, idx2, 32, 1.0, ws=ws)
+    assert kd.read_device_status(ws) == kd.KD_OK
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """A wait on a barrier nothing arrives at returns KD_ERR_TIMEOUT by itself."""
+    require_gpu()
+    ws = kd.alloc_workspace(4096, "cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    assert kd.kd_debug_wait_probe(ws.data_ptr(), ws.numel(), 2_000_000, st) == kd.KD_OK
+    assert kd.read_device_status(ws) == kd.KD_ERR_TIMEOUT
+    r = _run(128, 64, 1000, 8, 64, torch.bfloat16)          # the context still works
+    _full_parity(r)
+
+
+def test_autograd_function():
+    require_gpu()
+    h, W, vals, idx = inputs.make_loss_inputs(96, 64, 777, 10, dtype=torch.bfloat16, seed=2, device="cuda")
+    h.requires_grad_(True)
+    W.requires_grad_(True)
+    loss = kd.FusedTopKKLLoss.apply(h, W, vals, idx, 40, 1.0)
+    (2.0 * loss).backward()
+    torch.cuda.synchronize()
+    hn, Wn = to_np_exact(h), to_np_exact(W)
+    dH, dW = oracle.backward(hn, Wn, vals.cpu().numpy(), idx.cpu().numpy(), 1.0, 2.0)
+    assert rel_maxabs(h.grad.float().cpu().numpy(), dH) <= GRAD_TOL
+    assert rel_maxabs(W.grad.float().cpu().numpy(), dW) <= GRAD_TOL
+
+
+# ------------------------------------------------------------------ full-size
+
+def _sampled_full_size(name, n_rows, n_vrows=0):
+    cfg = inputs.WORKLOADS[name]
+    T, d, V, K, chunk = cfg["T"], cfg["d"], cfg["V"], cfg["K"], cfg["chunk"]
+    r = _run(T, d, V, K, chunk, torch.bfloat16)
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.choice(T, n_rows, replace=False))
+    rows[0] = 0
+    rows[-1] = T - 1                                 # both ends of the last (ragged) chunk
+    hn, Wn = to_np_exact(r["h"]), to_np_exact(r["W"])
+    vals, idx = r["vals"].cpu().numpy(), r["idx"].cpu().numpy()
+    lse_o, kl_o = oracle.forward_rows(hn, Wn, vals, idx, 1.0, rows)
+    assert np.abs(r["lse"].cpu().numpy()[rows] - lse_o).max() <= 1e-3
+    assert np.abs(r["kl"].cpu().numpy()[rows] - kl_o).max() <= 1e-2
+    dH_o = oracle.backward_dH_rows(hn, Wn, vals, idx, 1.0, rows, T)
+    assert rel_maxabs(r["dH"].float().cpu().numpy()[rows], dH_o) <= GRAD_TOL
+    # the loss is the mean of the per-row KL (checked above on sampled rows)
+    kl_all = r["kl"].cpu().numpy().astype(np.float64)
+    assert abs(r["loss"].item() - kl_all.mean()) <= 1e-6 * abs(kl_all.mean())
+    # zero-sum invariant: sum_v dz = 0 (S = 1) => sum_v dW[v, :] = 0
+    dW = r["dW"]
+    colsum = dW.double().sum(dim=0).abs().max().item()
+    assert colsum <= 1e-3 * dW.abs().max().item() * math.sqrt(V)
+    return r
+
+
+def test_toy_head_8k_sampled():
+    """T=8192, d=4096, V=131072, K=100, chunk=1024 (bench launch config)."""
+    require_gpu()
+    _sampled_full_size("head-8k", 32)
+
+
+@pytest.mark.slow
+def test_toy_head_32k_sampled():
+    """T=32768, d=4096, V=131072, K=100, chunk=2048 (the headline workload)."""
+    require_gpu()
+    _sampled_full_size("head-32k", 24)
+
+
+def test_dW_sampled_vocab_rows_full_width():
+    """Full d and V with a short T so the oracle's all-row LSE stays cheap:
+    T=384, d=4096, V=131072, K=100, chunk=256; 48 vocabulary rows of dW
+    (including every teacher index of row 0)."""
+    require_gpu()
+    T, d, V, K, chunk = 384, 4096, 131072, 100, 256
+    r = _run(T, d, V, K, chunk, torch.bfloat16)
+    hn, Wn = to_np_exact(r["h"]), to_np_exact(r["W"])
+    vals, idx = r["vals"].cpu().numpy(), r["idx"].cpu().numpy()
+    vrows = np.unique(np.concatenate([idx[0, :24], np.random.default_rng(2).choice(V, 24, replace=False),
+                                      [0, V - 1]]))
+    dW_o = oracle.backward_dW_rows(hn, Wn, vals, idx, 1.0, vrows)
+    assert rel_maxabs(r["dW"].cpu().numpy()[vrows], dW_o) <= GRAD_TOL
+    loss_o, _, _ = oracle.forward(hn, Wn, vals, idx, 1.0)
+    assert abs(r["loss"].item() - loss_o) <= LOSS_RTOL * abs(loss_o)
