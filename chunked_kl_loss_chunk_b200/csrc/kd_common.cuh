@@ -196,16 +196,23 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 // ----------------------------------------------------------------------------
 // UMMA shared-memory descriptor (sm_100 format): start>>4 in [0,14),
 // leading-byte-offset>>4 in [16,30), stride-byte-offset>>4 in [32,46),
-// version 1 at bit 46, layout type in [61,64) (2 = 128-byte swizzle).
+// version 1 at bit 46, layout type in [61,64).  Layout types used here:
+//   2 = 128-byte swizzle of 16-byte chunks over 8 rows of 128 bytes (K-major
+//       operands, and MN-major 16-bit operands);
+//   1 = 128-byte swizzle of 32-byte chunks over 4 rows of 128 bytes (the only
+//       layout the tensor cores accept for MN-major tf32 operands).
 // ----------------------------------------------------------------------------
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr, uint32_t lbo_bytes,
-                                                    uint32_t sbo_bytes) {
+constexpr uint64_t UMMA_LAYOUT_SW128 = 2;
+constexpr uint64_t UMMA_LAYOUT_SW128_ATOM32 = 1;
+
+__device__ __forceinline__ uint64_t umma_desc(uint32_t smem_addr, uint32_t lbo_bytes,
+                                              uint32_t sbo_bytes, uint64_t layout) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
   d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
   d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= 1ull << 46;
-  d |= 2ull << 61;
+  d |= layout << 61;
   return d;
 }
 

@@ -40,12 +40,18 @@ struct ElemCfg<__nv_bfloat16> {
   static constexpr int BK = 64;        // elements per 128-byte row
   static constexpr int UMMA_K = 16;    // K per MMA instruction
   static constexpr uint32_t FMT = 1;   // bf16
+  // MN-major operands: 128-byte swizzle, 8-row atoms of 1024 bytes
+  static constexpr uint64_t MN_LAYOUT = UMMA_LAYOUT_SW128;
+  static constexpr uint32_t MN_SBO = 1024;
 };
 template <>
 struct ElemCfg<float> {
   static constexpr int BK = 32;
   static constexpr int UMMA_K = 8;
   static constexpr uint32_t FMT = 2;   // tf32
+  // MN-major tf32 operands: 128-byte swizzle with 32-byte chunks, 4-row atoms
+  static constexpr uint64_t MN_LAYOUT = UMMA_LAYOUT_SW128_ATOM32;
+  static constexpr uint32_t MN_SBO = 512;
 };
 
 enum EpiKind : int { EPI_FWD_LSE = 0, EPI_BWD_DZ = 1, EPI_STORE_H = 2, EPI_ACCUM_W = 3 };
@@ -370,10 +376,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
           for (int k = 0; k < KSTEPS; ++k) {
             // K-major: advance 32 bytes inside the swizzled row (SBO = 8 rows);
             // MN-major: advance UMMA_K rows (LBO = next MN box, SBO = 8 rows).
-            const uint64_t ad = A_MN ? umma_desc_sw128(a0 + k * C::UMMA_K * ROW_BYTES, BOX_BYTES, 1024)
-                                     : umma_desc_sw128(a0 + k * 32, 16, 1024);
-            const uint64_t bd = B_MN ? umma_desc_sw128(b0 + k * C::UMMA_K * ROW_BYTES, BOX_BYTES, 1024)
-                                     : umma_desc_sw128(b0 + k * 32, 16, 1024);
+            const uint64_t ad =
+                A_MN ? umma_desc(a0 + k * C::UMMA_K * ROW_BYTES, BOX_BYTES, C::MN_SBO, C::MN_LAYOUT)
+                     : umma_desc(a0 + k * 32, 16, 1024, UMMA_LAYOUT_SW128);
+            const uint64_t bd =
+                B_MN ? umma_desc(b0 + k * C::UMMA_K * ROW_BYTES, BOX_BYTES, C::MN_SBO, C::MN_LAYOUT)
+                     : umma_desc(b0 + k * 32, 16, 1024, UMMA_LAYOUT_SW128);
             const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
             if constexpr (C::FMT == 1) mma_f16(d_tmem, ad, bd, IDESC, accum);
             else mma_tf32(d_tmem, ad, bd, IDESC, accum);

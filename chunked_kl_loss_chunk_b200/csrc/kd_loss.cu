@@ -203,9 +203,12 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2-D row-major tensor [outer, inner] with the given row pitch (elements),
-// 128-byte swizzle, zero fill out of bounds.
+// zero fill out of bounds.  Swizzle: 128 bytes of 16-byte chunks, except for
+// fp32 tiles read MN-major by the tensor cores (mn_major && f32), which need
+// 128 bytes of 32-byte chunks to match the MMA's tf32 MN-major layout.
 bool make_map(CUtensorMap* map, const void* base, bool f32, uint64_t inner, uint64_t outer,
-              uint64_t pitch_elems, uint32_t box_inner, uint32_t box_outer) {
+              uint64_t pitch_elems, uint32_t box_inner, uint32_t box_outer,
+              bool mn_major = false) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const uint64_t es = f32 ? 4 : 2;
@@ -215,7 +218,8 @@ bool make_map(CUtensorMap* map, const void* base, bool f32, uint64_t inner, uint
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                   2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  (mn_major && f32) ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -362,7 +366,7 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
   }
   CUtensorMap tW_k, tW_mn;
   if (!make_map(&tW_k, W, F32, d, V, d, BK, BN)) return KD_ERR_CUDA;      // [V, d], K = d
-  if (!make_map(&tW_mn, W, F32, d, V, d, INNER, BK)) return KD_ERR_CUDA;  // K = V rows, N = d
+  if (!make_map(&tW_mn, W, F32, d, V, d, INNER, BK, true)) return KD_ERR_CUDA;  // K = V, N = d
   const float zscale = 1.4426950408889634f * inv_tau;
   const float inv_T_tau = static_cast<float>(1.0 / (static_cast<double>(T) * tau));
   for (int64_t c0 = 0; c0 < T; c0 += chunk) {
@@ -370,9 +374,9 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     const Elem* hc = static_cast<const Elem*>(h) + c0 * d;
     CUtensorMap tH_k, tH_mn, tDz_k, tDz_mn;
     if (!make_map(&tH_k, hc, F32, d, rows, d, BK, BM)) return KD_ERR_CUDA;
-    if (!make_map(&tH_mn, hc, F32, d, rows, d, INNER, BK)) return KD_ERR_CUDA;
+    if (!make_map(&tH_mn, hc, F32, d, rows, d, INNER, BK, true)) return KD_ERR_CUDA;
     if (!make_map(&tDz_k, dz, F32, V, rows, L.ldz, BK, BM)) return KD_ERR_CUDA;
-    if (!make_map(&tDz_mn, dz, F32, V, rows, L.ldz, INNER, BK)) return KD_ERR_CUDA;
+    if (!make_map(&tDz_mn, dz, F32, V, rows, L.ldz, INNER, BK, true)) return KD_ERR_CUDA;
 
     // (1) recompute z = h_c W^T; epilogue writes dz_c [rows, ldz]
     GemmArgs g;

@@ -195,8 +195,11 @@ def _ptr(t):
 
 
 def alloc_workspace(nbytes: int, device) -> torch.Tensor:
-    """Caller-owned workspace (1024-byte aligned by the caching allocator)."""
-    ws = torch.empty(max(int(nbytes), 1024), dtype=torch.uint8, device=device)
+    """Caller-owned workspace: a 1024-byte-aligned uint8 view of ``nbytes``."""
+    n = max(int(nbytes), 1024)
+    buf = torch.empty(n + 1024, dtype=torch.uint8, device=device)
+    off = (-buf.data_ptr()) % 1024
+    ws = buf[off:off + n]
     assert ws.data_ptr() % 1024 == 0
     return ws
 
