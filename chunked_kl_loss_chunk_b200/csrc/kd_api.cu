@@ -38,6 +38,8 @@ namespace kd {
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+uint64_t wait_limit_ns() { return g_wait_limit_ns; }
+
 void profile_before(int kind, double flops, cudaStream_t s) {
   g_prof.armed = false;
   if (!g_prof.start || !(g_prof.mask & kind) || g_prof.n >= g_prof.capacity) return;

@@ -32,6 +32,9 @@ cudaError_t launch_topk_bf16(const void* logits, int64_t T, int64_t V, int K, fl
 
 cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
 
+// Current time limit of device-side waits (kd_set_wait_limit_ns).
+uint64_t wait_limit_ns();
+
 // Launch accounting and optional per-GEMM event recording.
 void count_launch();
 void profile_before(int kind, double flops, cudaStream_t s);

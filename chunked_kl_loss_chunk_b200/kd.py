@@ -44,6 +44,8 @@ _SIGNATURES = {
     "kd_set_wait_limit_ns": (_c_int, [_c_u64]),
     "kd_debug_wait_probe": (_c_int, [_c_vp, _c_sz, _c_u64, _c_vp]),
     "kd_launch_count": (_c_u64, []),
+    "kd_fused_kl_fwd_noalloc": (_c_int, [_c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp,
+                                         _c_int, _c_i64, ctypes.c_float, _c_vp, _c_vp, _c_vp, _c_vp]),
     "kd_profile_attach": (_c_int, [_c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_int]),
     "kd_profile_detach": (_c_int, []),
 }
@@ -116,6 +118,14 @@ def kd_fused_kl_bwd(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, 
                     dW, accumulate_dW, ws, ws_bytes, stream):
     return load().kd_fused_kl_bwd(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, lse,
                                   grad_loss, dH, dW, accumulate_dW, ws, ws_bytes, stream)
+
+
+def kd_fused_kl_fwd_noalloc(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, loss, lse,
+                            kl_rows, stream):
+    """Forward for callers that cannot provide a workspace (scratch is a fixed
+    array inside the library; see include/kd.h for its limit and caveats)."""
+    return load().kd_fused_kl_fwd_noalloc(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature,
+                                          loss, lse, kl_rows, stream)
 
 
 def kd_read_device_status(ws, stream):

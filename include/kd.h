@@ -157,6 +157,41 @@ kd_status kd_set_wait_limit_ns(uint64_t limit_ns);
 kd_status kd_debug_wait_probe(void* ws, size_t ws_bytes, uint64_t limit_ns, void* stream);
 
 /* ------------------------------------------------------------------------ */
+/* Forward without a caller workspace.  (The pages have no counterpart to   */
+/* this entry point; it exists for callers of this library.)                */
+/* ------------------------------------------------------------------------ */
+
+/* Size of the scratch array compiled into the library for
+ * kd_fused_kl_fwd_noalloc.  Every GPU that loads the library holds this much
+ * device memory until the process exits. */
+#define KD_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/*
+ * Same computation, arguments and outputs as kd_fused_kl_fwd, for callers that
+ * cannot provide a workspace -- for example a plugin that receives only its
+ * input and output pointers, or a program whose device memory all belongs to
+ * another framework's pool.  Scratch comes from a fixed array inside the
+ * library; nothing is allocated.
+ *   - Scratch needed: about 8*T*K + 12*T + 16*min(chunk,T)*ceil(V/256) bytes
+ *     plus alignment; when that exceeds KD_NOALLOC_SCRATCH_BYTES the call
+ *     returns KD_ERR_WORKSPACE and launches nothing (e.g. T=32768, K=100,
+ *     chunk=2048, V=131072 needs about 43 MB and fits).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls share the one array: calls that can overlap on the GPU (other
+ *     streams, other threads) race and give wrong results; serialise them.
+ *   - Device-side status (bad cache index, timeout) goes to the array's status
+ *     word, which this ABI does not expose; use kd_fused_kl_fwd with a
+ *     workspace when that check matters.
+ */
+kd_status kd_fused_kl_fwd_noalloc(const void* h, const void* W, int dtype,
+                                  int64_t T, int64_t d, int64_t V,
+                                  const float* t_vals, const int32_t* t_idx, int K,
+                                  int64_t chunk, float temperature,
+                                  float* loss, float* lse, float* kl_rows, void* stream);
+
+/* ------------------------------------------------------------------------ */
 /* Measurement support (process-wide state; not thread-safe).              */
 /* ------------------------------------------------------------------------ */
 
