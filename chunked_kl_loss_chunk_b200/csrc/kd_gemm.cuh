@@ -31,7 +31,11 @@ constexpr int A_STAGE_BYTES = BM * ROW_BYTES;  // 16 KB
 constexpr int B_STAGE_BYTES = BN * ROW_BYTES;  // 32 KB
 constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int TMEM_COLS = 2 * BN;              // two accumulators
-constexpr int GEMM_SMEM_BYTES = STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+constexpr int EPI_WARPS = 4;
+constexpr int EPI_BUF_BYTES = 32 * 128;        // one 32x32 fp32 (or 32x32 bf16) output box
+constexpr int EPI_SMEM_BYTES = EPI_WARPS * 2 * EPI_BUF_BYTES;   // double-buffered per warp
+constexpr int GEMM_SMEM_BYTES =
+    STAGES * STAGE_BYTES + EPI_SMEM_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
 template <typename Elem>
 struct ElemCfg;
@@ -79,27 +83,58 @@ struct GemmArgs {
   uint64_t wait_limit_ns;
 };
 
-template <typename Elem>
-__device__ __forceinline__ void store8(Elem* dst, const float* v);
-
-template <>
-__device__ __forceinline__ void store8<__nv_bfloat16>(__nv_bfloat16* dst, const float* v) {
-  uint4 q;
-  __nv_bfloat162 a = __floats2bfloat162_rn(v[0], v[1]);
-  __nv_bfloat162 b = __floats2bfloat162_rn(v[2], v[3]);
-  __nv_bfloat162 c = __floats2bfloat162_rn(v[4], v[5]);
-  __nv_bfloat162 d = __floats2bfloat162_rn(v[6], v[7]);
-  q.x = *reinterpret_cast<uint32_t*>(&a);
-  q.y = *reinterpret_cast<uint32_t*>(&b);
-  q.z = *reinterpret_cast<uint32_t*>(&c);
-  q.w = *reinterpret_cast<uint32_t*>(&d);
-  *reinterpret_cast<uint4*>(dst) = q;
+// ----------------------------------------------------------------------------
+// Output boxes.  An epilogue warp owns 32 accumulator rows; every 32-column
+// block of its rows is converted, written to a shared-memory box in the TMA
+// swizzle of the output tensor map, and sent out by one lane with a TMA store
+// (or, for accumulating fp32 output, a TMA add-reduction).  Two boxes per warp
+// alternate so that writing one overlaps the transfer of the other.
+//   fp32 box: 32 rows x 128 B, 128-byte swizzle (16-byte chunk j of row r at
+//             chunk j ^ (r & 7));
+//   bf16 box: 32 rows x  64 B,  64-byte swizzle (chunk j of row r at
+//             chunk j ^ ((r >> 1) & 3)).
+// Both layouts spread a warp's 16-byte writes over all 32 banks.
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ void stage_box_f32(unsigned char* box, int r, const float* v) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<float4*>(box + r * 128 + ((j ^ (r & 7)) << 4)) =
+        make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
 }
 
-template <>
-__device__ __forceinline__ void store8<float>(float* dst, const float* v) {
-  reinterpret_cast<float4*>(dst)[0] = make_float4(v[0], v[1], v[2], v[3]);
-  reinterpret_cast<float4*>(dst)[1] = make_float4(v[4], v[5], v[6], v[7]);
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&b);
+}
+
+__device__ __forceinline__ void stage_box_bf16(unsigned char* box, int r, const float* v) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint4 q;
+    q.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+    q.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+    q.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+    q.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+    *reinterpret_cast<uint4*>(box + r * 64 + ((j ^ ((r >> 1) & 3)) << 4)) = q;
+  }
+}
+
+// Hands one staged box to TMA.  Called by every lane of the warp.
+template <typename OutT>
+__device__ __forceinline__ void emit_box(const CUtensorMap* tmC, unsigned char* box, int x, int y,
+                                         bool reduce_add) {
+  fence_proxy_async_smem();
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) {
+    if (reduce_add) tma_reduce_add_2d(tmC, box, x, y); else tma_store_2d(tmC, box, x, y);
+    bulk_commit();
+  }
+}
+
+// Before reusing a box: the transfer issued from it two blocks ago has read it.
+__device__ __forceinline__ void box_reuse_wait() {
+  if ((threadIdx.x & 31) == 0) bulk_wait_read<1>();
+  __syncwarp();
 }
 
 // First position in the ascending list ids[0..K) holding a value >= key.
@@ -114,15 +149,19 @@ __device__ __forceinline__ int lower_bound_i32(const int32_t* ids, int K, int32_
 
 // ----------------------------------------------------------------------------
 // Epilogues.  Called by the 128 epilogue threads; `taddr` addresses this
-// warp's 32 TMEM lanes at the tile's first accumulator column.  Every thread
-// of a warp executes the same sequence of tcgen05.ld (they are warp-collective).
+// warp's 32 TMEM lanes at the tile's first accumulator column; `boxes` is the
+// warp's pair of output boxes.  Every lane of a warp executes the same sequence
+// of tcgen05.ld (they are warp-collective).
 // ----------------------------------------------------------------------------
 template <typename Elem, int EPI>
-__device__ __forceinline__ void run_epilogue(const GemmArgs& g, int mb, int nb, uint32_t taddr,
-                                             int r) {
+__device__ __forceinline__ void run_epilogue(const GemmArgs& g, const CUtensorMap* tmC, int mb,
+                                             int nb, uint32_t taddr, int quad, int lane,
+                                             unsigned char* boxes) {
+  const int r = quad * 32 + lane;         // accumulator row of this thread
   const int m = mb * BM + r;              // output row within the problem
   const bool row_ok = m < g.M;
   const int n0 = nb * BN;
+  const int y_box = mb * BM + quad * 32;  // first output row of this warp's boxes
 
   if constexpr (EPI == EPI_FWD_LSE || EPI == EPI_BWD_DZ) {
     const int64_t t = g.row0 + m;         // global position
@@ -174,7 +213,7 @@ __device__ __forceinline__ void run_epilogue(const GemmArgs& g, int mb, int nb, 
       }
       if (row_ok) g.partials[static_cast<int64_t>(m) * g.n_tiles + nb] =
           make_float4(run_m, run_s, gat, 0.f);
-    } else {  // EPI_BWD_DZ
+    } else {  // EPI_BWD_DZ: dz box per 32 columns; TMA clips columns >= V, rows >= M
       const float gl = g.grad_loss ? __ldg(g.grad_loss) : 1.f;
       const float coef = gl * g.inv_T_tau;
       float coefA = 0.f, off = 0.f;
@@ -182,13 +221,13 @@ __device__ __forceinline__ void run_epilogue(const GemmArgs& g, int mb, int nb, 
         coefA = coef * g.row_stats[t].x;
         off = -__ldg(g.lse + t) * 1.4426950408889634f;   // -LSE * log2(e)
       }
-      Elem* dst = static_cast<Elem*>(g.out) + static_cast<int64_t>(m) * g.ldo;
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         const int base = n0 + c * 32;
         if (base >= g.V) break;
+        unsigned char* box = boxes + (c & 1) * EPI_BUF_BYTES;
+        box_reuse_wait();
         float v[32];
-        __syncwarp();
         tmem_ld32(taddr + c * 32, v);
 #pragma unroll
         for (int j = 0; j < 32; ++j) v[j] = coefA * ex2_approx(fmaf(v[j], zs, off));
@@ -203,51 +242,23 @@ __device__ __forceinline__ void run_epilogue(const GemmArgs& g, int mb, int nb, 
             }
           }
         }
-        if (base + 32 > g.V) {
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (base + j >= g.V) v[j] = 0.f;
-        }
-        if (row_ok) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) store8<Elem>(dst + base + 8 * u, v + 8 * u);
-        }
+        if constexpr (sizeof(Elem) == 4) stage_box_f32(box, lane, v);
+        else stage_box_bf16(box, lane, v);
+        emit_box<Elem>(tmC, box, base, y_box, false);
       }
     }
-  } else if constexpr (EPI == EPI_STORE_H) {
-    Elem* dst = static_cast<Elem*>(g.out) + (g.row0 + m) * g.ldo;
+  } else {  // EPI_STORE_H (dtype of h) or EPI_ACCUM_W (fp32, store or add)
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
       const int base = n0 + c * 32;
       if (base >= g.N) break;
+      unsigned char* box = boxes + (c & 1) * EPI_BUF_BYTES;
+      box_reuse_wait();
       float v[32];
-      __syncwarp();
       tmem_ld32(taddr + c * 32, v);
-      if (row_ok) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (base + 8 * u < g.N) store8<Elem>(dst + base + 8 * u, v + 8 * u);
-      }
-    }
-  } else {  // EPI_ACCUM_W: fp32 dW rows, N % 4 == 0
-    float* dst = static_cast<float*>(g.out) + static_cast<int64_t>(m) * g.ldo;
-#pragma unroll 1
-    for (int c = 0; c < BN / 32; ++c) {
-      const int base = n0 + c * 32;
-      if (base >= g.N) break;
-      float v[32];
-      __syncwarp();
-      tmem_ld32(taddr + c * 32, v);
-      if (row_ok) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (base + 4 * u < g.N) {
-            float4* p = reinterpret_cast<float4*>(dst + base + 4 * u);
-            const float4 x = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-            if (g.accumulate) atomicAdd(p, x); else *p = x;
-          }
-        }
-      }
+      if constexpr (EPI == EPI_STORE_H && sizeof(Elem) == 2) stage_box_bf16(box, lane, v);
+      else stage_box_f32(box, lane, v);
+      emit_box<Elem>(tmC, box, base, y_box, EPI == EPI_ACCUM_W && g.accumulate);
     }
   }
 }
@@ -258,7 +269,7 @@ __device__ __forceinline__ void run_epilogue(const GemmArgs& g, int mb, int nb, 
 template <typename Elem, int A_MN, int B_MN, int EPI>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-            const GemmArgs g) {
+            const __grid_constant__ CUtensorMap tmC, const GemmArgs g) {
   using C = ElemCfg<Elem>;
   constexpr int BK = C::BK;
   constexpr int INNER = ROW_BYTES / sizeof(Elem);        // MN elements per MN-major box
@@ -271,7 +282,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   unsigned char* sA = smem;
   unsigned char* sB = smem + STAGES * A_STAGE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  unsigned char* sEpi = smem + STAGES * STAGE_BYTES;      // [EPI_WARPS][2][EPI_BUF_BYTES]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + EPI_SMEM_BYTES);
   uint64_t* full = bars;                 // [STAGES]
   uint64_t* empty = bars + STAGES;       // [STAGES]
   uint64_t* tfull = bars + 2 * STAGES;   // [2]
@@ -296,6 +308,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    if (EPI != EPI_FWD_LSE) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, TMEM_COLS);
@@ -407,7 +420,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
   } else {
     // ------------------------------------------------------------ epilogue
     const int quad = warp & 3;                 // TMEM lane quadrant of this warp
-    const int r = quad * 32 + lane;            // accumulator row of this thread
+    unsigned char* boxes = sEpi + (warp - 2) * 2 * EPI_BUF_BYTES;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -417,7 +430,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      run_epilogue<Elem, EPI>(g, mb, nb, taddr, r);
+      run_epilogue<Elem, EPI>(g, &tmC, mb, nb, taddr, quad, lane, boxes);
       __syncwarp();
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
@@ -426,6 +439,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
         acc_phase ^= 1u;
       }
     }
+    // Every output box must have left shared memory and landed before exit.
+    if (lane == 0) bulk_wait<0>();
+    __syncwarp();
   }
 
   tc_fence_before();

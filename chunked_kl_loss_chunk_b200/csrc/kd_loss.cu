@@ -208,7 +208,7 @@ EncodeTiledFn encode_fn() {
 // 128 bytes of 32-byte chunks to match the MMA's tf32 MN-major layout.
 bool make_map(CUtensorMap* map, const void* base, bool f32, uint64_t inner, uint64_t outer,
               uint64_t pitch_elems, uint32_t box_inner, uint32_t box_outer,
-              bool mn_major = false) {
+              bool mn_major = false, int swizzle_override = -1) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const uint64_t es = f32 ? 4 : 2;
@@ -219,14 +219,24 @@ bool make_map(CUtensorMap* map, const void* base, bool f32, uint64_t inner, uint
   CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                   2, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  (mn_major && f32) ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B,
+                  swizzle_override >= 0 ? static_cast<CUtensorMapSwizzle>(swizzle_override)
+                  : (mn_major && f32)   ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
+                                        : CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
+// Output box map for the epilogues: 32 x 32 elements, 128-byte swizzle for
+// fp32 boxes (128-byte rows), 64-byte swizzle for bf16 boxes (64-byte rows).
+bool make_out_map(CUtensorMap* map, const void* base, bool f32, uint64_t inner, uint64_t outer,
+                  uint64_t pitch_elems) {
+  return make_map(map, base, f32, inner, outer, pitch_elems, 32, 32, false,
+                  f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
 template <typename Elem, int A_MN, int B_MN, int EPI>
-cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmArgs g,
-                        cudaStream_t s, int num_sms) {
+cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
+                        GemmArgs g, cudaStream_t s, int num_sms) {
   static constexpr int kKind[4] = {KD_GEMM_FWD_LSE, KD_GEMM_BWD_DZ, KD_GEMM_DH, KD_GEMM_DW};
   auto kern = gemm_kernel<Elem, A_MN, B_MN, EPI>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -235,7 +245,7 @@ cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, GemmArgs g
   const int tiles = g.m_tiles * g.n_tiles;
   const int grid = tiles < num_sms ? tiles : num_sms;
   profile_before(kKind[EPI], 2.0 * g.M * static_cast<double>(g.N) * g.K, s);
-  kern<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, s>>>(ta, tb, g);
+  kern<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, s>>>(ta, tb, tc, g);
   count_launch();
   profile_after(s);
   return cudaGetLastError();
@@ -323,7 +333,8 @@ static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     g.partials = part;
     g.status = status;
     g.wait_limit_ns = limit_ns;
-    if (launch_gemm<Elem, 0, 0, EPI_FWD_LSE>(tH, tW, g, s, num_sms) != cudaSuccess)
+    if (launch_gemm<Elem, 0, 0, EPI_FWD_LSE>(tH, tW, tH /*no output box*/, g, s, num_sms) !=
+        cudaSuccess)
       return KD_ERR_CUDA;
     const int cblocks = cdiv(rows * 32, 256);
     combine_kernel<<<cblocks, 256, 0, s>>>(part, static_cast<int>(rows), g.n_tiles, c0, zscale,
@@ -367,12 +378,17 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
   CUtensorMap tW_k, tW_mn;
   if (!make_map(&tW_k, W, F32, d, V, d, BK, BN)) return KD_ERR_CUDA;      // [V, d], K = d
   if (!make_map(&tW_mn, W, F32, d, V, d, INNER, BK, true)) return KD_ERR_CUDA;  // K = V, N = d
+  CUtensorMap tDW_out;
+  if (!make_out_map(&tDW_out, dW, true, d, V, d)) return KD_ERR_CUDA;
   const float zscale = 1.4426950408889634f * inv_tau;
   const float inv_T_tau = static_cast<float>(1.0 / (static_cast<double>(T) * tau));
   for (int64_t c0 = 0; c0 < T; c0 += chunk) {
     const int64_t rows = (T - c0) < chunk ? (T - c0) : chunk;
     const Elem* hc = static_cast<const Elem*>(h) + c0 * d;
-    CUtensorMap tH_k, tH_mn, tDz_k, tDz_mn;
+    CUtensorMap tH_k, tH_mn, tDz_k, tDz_mn, tDz_out, tDH_out;
+    if (!make_out_map(&tDz_out, dz, F32, V, rows, L.ldz)) return KD_ERR_CUDA;
+    if (!make_out_map(&tDH_out, static_cast<Elem*>(dH) + c0 * d, F32, d, rows, d))
+      return KD_ERR_CUDA;
     if (!make_map(&tH_k, hc, F32, d, rows, d, BK, BM)) return KD_ERR_CUDA;
     if (!make_map(&tH_mn, hc, F32, d, rows, d, INNER, BK, true)) return KD_ERR_CUDA;
     if (!make_map(&tDz_k, dz, F32, V, rows, L.ldz, BK, BM)) return KD_ERR_CUDA;
@@ -402,7 +418,7 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     g.ldo = L.ldz;
     g.status = status;
     g.wait_limit_ns = limit_ns;
-    if (launch_gemm<Elem, 0, 0, EPI_BWD_DZ>(tH_k, tW_k, g, s, num_sms) != cudaSuccess)
+    if (launch_gemm<Elem, 0, 0, EPI_BWD_DZ>(tH_k, tW_k, tDz_out, g, s, num_sms) != cudaSuccess)
       return KD_ERR_CUDA;
 
     // (2) dH_c = dz_c W : M = rows, N = d, K = V; A K-major, B MN-major
@@ -414,7 +430,8 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     gh.m_fastest = 1;
     gh.out = dH;
     gh.ldo = d;
-    if (launch_gemm<Elem, 0, 1, EPI_STORE_H>(tDz_k, tW_mn, gh, s, num_sms) != cudaSuccess)
+    if (launch_gemm<Elem, 0, 1, EPI_STORE_H>(tDz_k, tW_mn, tDH_out, gh, s, num_sms) !=
+        cudaSuccess)
       return KD_ERR_CUDA;
 
     // (3) dW (+)= dz_c^T h_c : M = V, N = d, K = rows; both operands MN-major
@@ -430,7 +447,8 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     gw.out = dW;
     gw.ldo = d;
     gw.accumulate = (accumulate || c0 > 0) ? 1 : 0;
-    if (launch_gemm<Elem, 1, 1, EPI_ACCUM_W>(tDz_mn, tH_mn, gw, s, num_sms) != cudaSuccess)
+    if (launch_gemm<Elem, 1, 1, EPI_ACCUM_W>(tDz_mn, tH_mn, tDW_out, gw, s, num_sms) !=
+        cudaSuccess)
       return KD_ERR_CUDA;
   }
   return KD_OK;

@@ -28,6 +28,7 @@ constexpr int TK_BINS = 4096;       // bins of (order key >> 4)
 constexpr int TK_SAMPLE = 4096;
 constexpr int TK_CAND_CAP = 2048;
 constexpr int TK_SEL_CAP = 1024;    // >= K
+constexpr int TK_UNROLL = 8;        // 16-byte loads in flight per thread
 
 // Order-preserving 16-bit key of a bf16 bit pattern: NaN -> 0 (lowest),
 // -0 -> key of +0, otherwise a monotone map of the value.
@@ -159,14 +160,26 @@ __device__ __forceinline__ void for_each_elem(const uint16_t* __restrict__ row, 
   for (int64_t i = threadIdx.x; i < head; i += TK_THREADS) f(row[i], static_cast<uint32_t>(i));
   const int64_t nvec = (V - head) >> 3;
   const uint4* vp = reinterpret_cast<const uint4*>(row + head);
-  for (int64_t j = threadIdx.x; j < nvec; j += TK_THREADS) {
-    const uint4 q = __ldcs(vp + j);
-    const uint32_t base = static_cast<uint32_t>(head + (j << 3));
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  // TK_UNROLL independent 16-byte loads in flight per thread before any use.
+  for (int64_t j0 = threadIdx.x; j0 < nvec; j0 += TK_THREADS * TK_UNROLL) {
+    uint4 q[TK_UNROLL];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      f(w[u] & 0xFFFFu, base + 2 * u);
-      f(w[u] >> 16, base + 2 * u + 1);
+    for (int u = 0; u < TK_UNROLL; ++u) {
+      const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
+      q[u] = j < nvec ? __ldcs(vp + j) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < TK_UNROLL; ++u) {
+      const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
+      if (j < nvec) {
+        const uint32_t base = static_cast<uint32_t>(head + (j << 3));
+        const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          f(w[e] & 0xFFFFu, base + 2 * e);
+          f(w[e] >> 16, base + 2 * e + 1);
+        }
+      }
     }
   }
   for (int64_t i = head + (nvec << 3) + threadIdx.x; i < V; i += TK_THREADS)

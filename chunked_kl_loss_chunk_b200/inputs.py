@@ -87,8 +87,9 @@ WORKLOADS = {
     "head-32k": dict(T=32768, d=4096, V=131072, K=100, chunk=2048, dtype="bf16"),
     "vocab-201k": dict(T=32768, d=2880, V=201088, K=100, chunk=2048, dtype="bf16"),
     "long-256k": dict(T=262144, d=4096, V=131072, K=100, chunk=4096, dtype="bf16"),
-    # one 2048-position chunk of the 32K head: a small case for kernel profiles
+    # one and two 2048-position chunks of the 32K head: small cases for profiles
     "head-2k": dict(T=2048, d=4096, V=131072, K=100, chunk=2048, dtype="bf16"),
+    "head-4k": dict(T=4096, d=4096, V=131072, K=100, chunk=2048, dtype="bf16"),
 }
 
 TOPK_WORKLOADS = {
