@@ -6,10 +6,11 @@
 // (value descending, index ascending), +0 == -0, NaN below -inf.
 //
 // Design (HBM-bound streaming select):
-//   1. sample: 4096-bin histogram (order key >> 4) of the first min(V, 4096)
-//      elements gives a threshold bin L whose count from the top covers about
-//      4K expected row elements.  L is turned into a float threshold tf with
-//      key(x) >= L<<4  <=>  x >= tf  for every non-NaN x.
+//   1. sample: a 4096-bin histogram (order key >> 4) of the first
+//      min(V, 4096) elements, refined inside the threshold bin, gives the key L
+//      of the sample element ranked ~3K*S/V from the top (about 3K expected
+//      survivors in the row).  L is turned into a float threshold tf with
+//      key(x) >= L  <=>  x >= tf  for every non-NaN x.
 //   2. stream: one coalesced 16-byte-vector pass over the row; each element is
 //      one float compare against tf; the rare survivors are appended to a
 //      shared-memory candidate buffer.
@@ -23,7 +24,7 @@
 
 namespace kd {
 
-constexpr int TK_THREADS = 512;
+constexpr int TK_THREADS = 256;
 constexpr int TK_BINS = 4096;       // bins of (order key >> 4)
 constexpr int TK_SAMPLE = 4096;
 constexpr int TK_CAND_CAP = 2048;
@@ -206,17 +207,38 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
     const int64_t S = V < TK_SAMPLE ? V : TK_SAMPLE;
     for (int64_t i = tid; i < S; i += TK_THREADS)
       atomicAdd(&sm.hist[bf16_order_key(row[i]) >> 4], 1u);
+    if (tid < 16) sm.hist16[tid] = 0u;
     __syncthreads();
     uint32_t target;
     if (S == V) {
       target = static_cast<uint32_t>(K);
     } else {
-      const double want = 4.0 * K * static_cast<double>(S) / static_cast<double>(V);
+      // about 3K expected survivors over the whole row
+      const double want = 3.0 * K * static_cast<double>(S) / static_cast<double>(V);
       target = static_cast<uint32_t>(ceil(want));
       if (target < 1u) target = 1u;
     }
     find_threshold_bin(sm, target);
-    const uint32_t L = sm.thr_bin << 4;   // candidate iff order key >= L
+    // Refine to the exact key of the target-th largest sample element: split
+    // the threshold bin into its 16 keys.
+    const uint32_t sb = sm.thr_bin, s_above = sm.thr_above;
+    for (int64_t i = tid; i < S; i += TK_THREADS) {
+      const uint32_t key = bf16_order_key(row[i]);
+      if ((key >> 4) == sb) atomicAdd(&sm.hist16[key & 15u], 1u);
+    }
+    __syncthreads();
+    uint32_t L = sb << 4;                 // candidate iff order key >= L
+    {
+      uint32_t above = s_above;
+      for (int j = 15; j >= 0; --j) {
+        above += sm.hist16[j];
+        if (above >= target) {
+          L = (sb << 4) | static_cast<uint32_t>(j);
+          break;
+        }
+      }
+    }
+    __syncthreads();
     // Float threshold equivalent on non-NaN values: key >= L <=> x >= tf.
     float tf = 0.f;
     bool take_all = false;
@@ -224,6 +246,8 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
       take_all = true;                              // threshold inside the NaN bin
     } else if (L <= 0x7Fu) {
       tf = -INFINITY;                               // every non-NaN value qualifies
+    } else if (L == 0x7FFFu) {
+      tf = 0.f;                                     // between -0's raw key and +0
     } else if (L < 0x8000u) {
       tf = bf16_bits_to_float((~L) & 0xFFFFu);      // the negative value with key L
     } else {

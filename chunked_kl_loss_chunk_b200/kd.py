@@ -51,7 +51,7 @@ _SIGNATURES = {
 }
 
 KD_GEMM_FWD_LSE, KD_GEMM_BWD_DZ, KD_GEMM_DH, KD_GEMM_DW = 1, 2, 4, 8
-GEMM_KIND_NAMES = {1: "fwd_lse", 2: "bwd_dz", 4: "dH", 8: "dW"}
+GEMM_KIND_NAMES = {1: "fwd_lse", 2: "bwd_dz", 4: "dH", 8: "dW", 12: "dH+dW"}
 
 _lib = None
 
