@@ -34,6 +34,24 @@ if ROOT not in sys.path:
 METRIC = "tokens/s & TFLOP/s (8TdV) fused top-K KL fwd+bwd; % BF16 tensor peak; peak mem"
 UNIT = "tokens/s"
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
+# ncu capture of launches shaped exactly like the bench's (profiles/
+# gemm_topk_head-4k.md), valid only for the GEMM sources with this digest; the
+# roofline's "traffic" is null for any other source.
+NCU_TRAFFIC = {
+    "source_sha256_16": "e4030b4e36bf3456",
+    "per_launch_bytes": {"fwd_lse": 1.113e9, "bwd_dz": 1.628e9, "dH": 2.486e9, "dW": 4.66e9},
+}
+
+
+def _gemm_source_digest():
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "chunked_kl_loss_chunk_b200", "csrc")
+    for f in ("kd_common.cuh", "kd_gemm.cuh", "kd_loss.cu"):
+        h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
 
 def _args():
     ap = argparse.ArgumentParser()
@@ -395,7 +413,10 @@ def run_kd(args, rank, world):
         "dense_logits_grid_bytes_fp32": int(T * V * 4),
         "roofline": {"bound": "tensor", "kernel": f"gemm_kernel ({dom[0]})",
                      "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
-                     "frac": achieved / peak_sus, "traffic": None,
+                     "frac": achieved / peak_sus,
+                     "traffic": (NCU_TRAFFIC["per_launch_bytes"].get(dom[0])
+                                 if _gemm_source_digest() == NCU_TRAFFIC["source_sha256_16"]
+                                 else None),
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel inside a long step)"},
         "gpu_launches": int(n_launch),
         "clocks": clocks,
