@@ -48,7 +48,7 @@ def _gemm_source_digest():
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "chunked_kl_loss_chunk_b200", "csrc")
-    for f in ("kd_common.cuh", "kd_gemm.cuh", "kd_loss.cu"):
+    for f in ("kd_common.cuh", "kd_gemm.cuh", "kd_gemm2.cuh", "kd_loss.cu"):
         h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()[:16]
 

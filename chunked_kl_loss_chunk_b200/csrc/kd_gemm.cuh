@@ -58,7 +58,13 @@ struct ElemCfg<float> {
   static constexpr uint32_t MN_SBO = 512;
 };
 
-enum EpiKind : int { EPI_FWD_LSE = 0, EPI_BWD_DZ = 1, EPI_STORE_H = 2, EPI_ACCUM_W = 3 };
+enum EpiKind : int {
+  EPI_FWD_LSE = 0,        // logsumexp / gather partials per (row, vocabulary tile)
+  EPI_BWD_DZ = 1,         // dz boxes
+  EPI_STORE_H = 2,        // dH boxes in the dtype of h
+  EPI_ACCUM_W = 3,        // fp32 dW boxes, stored or added
+  EPI_STORE_PARTIAL = 4   // fp32 boxes of one K-split's partial dH
+};
 
 struct GemmArgs {
   int32_t M, N, K;
@@ -79,6 +85,8 @@ struct GemmArgs {
   void* out;                  // dz [M, ldo] | dH rows | dW
   int64_t ldo;                // leading dimension of `out`, elements
   int32_t accumulate;         // dW: add into `out`
+  int32_t k_split;            // K ranges per output tile (1 = no split)
+  int32_t split_rows;         // EPI_STORE_PARTIAL: rows between consecutive splits' partials
   uint32_t* status;
   uint64_t wait_limit_ns;
 };
@@ -154,14 +162,14 @@ __device__ __forceinline__ int lower_bound_i32(const int32_t* ids, int K, int32_
 // of tcgen05.ld (they are warp-collective).
 // ----------------------------------------------------------------------------
 template <typename Elem, int EPI>
-__device__ __forceinline__ void run_epilogue(const GemmArgs& g, const CUtensorMap* tmC, int mb,
+__device__ __forceinline__ void run_epilogue(const GemmArgs& g, const CUtensorMap* tmC, int m_base,
                                              int nb, uint32_t taddr, int quad, int lane,
-                                             unsigned char* boxes) {
+                                             unsigned char* boxes, int y_extra = 0) {
   const int r = quad * 32 + lane;         // accumulator row of this thread
-  const int m = mb * BM + r;              // output row within the problem
+  const int m = m_base + r;               // output row within the problem
   const bool row_ok = m < g.M;
   const int n0 = nb * BN;
-  const int y_box = mb * BM + quad * 32;  // first output row of this warp's boxes
+  const int y_box = y_extra + m_base + quad * 32;  // first output row of this warp's boxes
 
   if constexpr (EPI == EPI_FWD_LSE || EPI == EPI_BWD_DZ) {
     const int64_t t = g.row0 + m;         // global position
@@ -247,7 +255,7 @@ __device__ __forceinline__ void run_epilogue(const GemmArgs& g, const CUtensorMa
         emit_box<Elem>(tmC, box, base, y_box, false);
       }
     }
-  } else {  // EPI_STORE_H (dtype of h) or EPI_ACCUM_W (fp32, store or add)
+  } else {  // EPI_STORE_H (dtype of h), EPI_STORE_PARTIAL (fp32) or EPI_ACCUM_W (fp32)
 #pragma unroll 1
     for (int c = 0; c < BN / 32; ++c) {
       const int base = n0 + c * 32;
@@ -430,7 +438,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUt
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      run_epilogue<Elem, EPI>(g, &tmC, mb, nb, taddr, quad, lane, boxes);
+      run_epilogue<Elem, EPI>(g, &tmC, mb * BM, nb, taddr, quad, lane, boxes);
       __syncwarp();
       tc_fence_before();
       mbar_arrive(&tempty[acc]);

@@ -9,10 +9,15 @@
 
 namespace kd {
 
+// Largest number of K-splits used for dH = dz W (its fp32 partials live in
+// the workspace).
+constexpr int KD_DH_MAX_SPLIT = 4;
+
 // Byte offsets of the regions of a fused-loss workspace.
 struct WsLayout {
-  size_t p_sorted = 0, idx_sorted = 0, stats = 0, kl = 0, scratch = 0, total = 0;
-  int64_t ldz = 0;  // row pitch (elements) of the dz scratch
+  size_t p_sorted = 0, idx_sorted = 0, stats = 0, kl = 0, scratch = 0, hpart = 0, total = 0;
+  int64_t ldz = 0;       // row pitch (elements) of the dz scratch
+  int64_t rows_pad = 0;  // chunk rows rounded up to 256 (rows per dH partial)
 };
 
 WsLayout ws_layout(int64_t T, int64_t d, int64_t V, int K, int64_t chunk, int dtype);

@@ -12,6 +12,7 @@
 #include <string.h>
 
 #include "kd_gemm.cuh"
+#include "kd_gemm2.cuh"
 #include "kd_internal.h"
 
 namespace kd {
@@ -152,6 +153,36 @@ combine_kernel(const float4* __restrict__ partials, int rows, int n_tiles, int64
   }
 }
 
+// dH rows of a chunk = sum over K-splits of the fp32 partials, in split order.
+// One thread per 4 consecutive elements (d % 8 == 0).
+template <typename Elem>
+__global__ void __launch_bounds__(256)
+dh_reduce_kernel(const float* __restrict__ part, int k_split, int64_t split_rows, int rows,
+                 int64_t d, Elem* __restrict__ dH) {
+  const int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t per_row = d / 4;
+  if (q >= static_cast<int64_t>(rows) * per_row) return;
+  const int64_t m = q / per_row, j = (q - m * per_row) * 4;
+  float4 acc = reinterpret_cast<const float4*>(part + m * d + j)[0];
+  for (int s = 1; s < k_split; ++s) {
+    const float4 x = reinterpret_cast<const float4*>(part + (s * split_rows + m) * d + j)[0];
+    acc.x += x.x;
+    acc.y += x.y;
+    acc.z += x.z;
+    acc.w += x.w;
+  }
+  if constexpr (sizeof(Elem) == 4) {
+    reinterpret_cast<float4*>(dH + m * d + j)[0] = acc;
+  } else {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 w;
+    w.x = *reinterpret_cast<uint32_t*>(&lo);
+    w.y = *reinterpret_cast<uint32_t*>(&hi);
+    reinterpret_cast<uint2*>(dH + m * d + j)[0] = w;
+  }
+}
+
 // Deterministic mean of kl[0..T): one block, fixed per-thread strides, fixed
 // tree; fp64 accumulation.
 __global__ void __launch_bounds__(1024)
@@ -234,6 +265,84 @@ bool make_out_map(CUtensorMap* map, const void* base, bool f32, uint64_t inner, 
                   f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
+// Clusters of two CTAs that can be resident at once for this kernel.
+template <typename Kern>
+int max_pair_clusters(Kern kern, int num_sms) {
+  static int cached_dev = -1, cached = 0;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev == cached_dev && cached > 0) return cached;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (num_sms / 2));
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = GEMM2_SMEM_BYTES;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = num_sms / 2;
+  }
+  cached_dev = dev;
+  cached = n;
+  return n;
+}
+
+template <typename Elem, int A_MN, int B_MN, int EPI>
+cudaError_t launch_gemm2(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
+                         GemmArgs g, cudaStream_t s, int num_sms) {
+  static constexpr int kKind[5] = {KD_GEMM_FWD_LSE, KD_GEMM_BWD_DZ, KD_GEMM_DH, KD_GEMM_DW,
+                                   KD_GEMM_DH};
+  auto kern = gemm2_kernel<Elem, A_MN, B_MN, EPI>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       GEMM2_SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int units = ((g.M + BM2 - 1) / BM2) * g.n_tiles * g.k_split;
+  const int maxc = max_pair_clusters(kern, num_sms);
+  const int nclusters = units < maxc ? units : maxc;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * nclusters);
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = GEMM2_SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  profile_before(kKind[EPI], 2.0 * g.M * static_cast<double>(g.N) * g.K, s);
+  e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, g);
+  count_launch();
+  profile_after(s);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// K-splits (1..KD_DH_MAX_SPLIT, never more than k_blocks) for dH that best
+// fill the pair clusters.
+int choose_dh_split(int units1, int nclusters, int k_blocks) {
+  int best = 1;
+  double best_eff = 0.0;
+  const int kmax = k_blocks < KD_DH_MAX_SPLIT ? k_blocks : KD_DH_MAX_SPLIT;
+  for (int k = 1; k <= kmax; ++k) {
+    const int u = units1 * k;
+    const int rounds = (u + nclusters - 1) / nclusters;
+    const double eff = static_cast<double>(u) / (static_cast<double>(rounds) * nclusters);
+    if (eff > best_eff + 0.01) {
+      best_eff = eff;
+      best = k;
+    }
+  }
+  return best;
+}
+
 template <typename Elem, int A_MN, int B_MN, int EPI>
 cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
                         GemmArgs g, cudaStream_t s, int num_sms) {
@@ -256,7 +365,6 @@ inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b)
 }  // namespace
 
 WsLayout ws_layout(int64_t T, int64_t d, int64_t V, int K, int64_t chunk, int dtype) {
-  (void)d;
   WsLayout L;
   const size_t es = dtype == KD_DTYPE_F32 ? 4 : 2;
   auto al = [](size_t x) { return (x + 1023) & ~static_cast<size_t>(1023); };
@@ -276,6 +384,9 @@ WsLayout ws_layout(int64_t T, int64_t d, int64_t V, int K, int64_t chunk, int dt
   const size_t dz = static_cast<size_t>(rows) * static_cast<size_t>(L.ldz) * es;
   L.scratch = off;
   off = al(off + (part > dz ? part : dz));
+  L.rows_pad = ((rows + 255) / 256) * 256;
+  L.hpart = off;
+  off = al(off + static_cast<size_t>(KD_DH_MAX_SPLIT) * L.rows_pad * static_cast<size_t>(d) * 4);
   L.total = off;
   return L;
 }
@@ -307,7 +418,7 @@ static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
   }
   CUtensorMap tW;
-  if (!make_map(&tW, W, F32, d, V, d, BK, BN)) return KD_ERR_CUDA;
+  if (!make_map(&tW, W, F32, d, V, d, BK, 128)) return KD_ERR_CUDA;
   const float zscale = 1.4426950408889634f * inv_tau;
   for (int64_t c0 = 0; c0 < T; c0 += chunk) {
     const int64_t rows = (T - c0) < chunk ? (T - c0) : chunk;
@@ -323,6 +434,7 @@ static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     g.n_tiles = cdiv(V, BN);
     g.k_blocks = cdiv(d, BK);
     g.m_fastest = 1;
+    g.k_split = 1;
     g.row0 = c0;
     g.V = V;
     g.Ktop = K;
@@ -333,7 +445,7 @@ static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     g.partials = part;
     g.status = status;
     g.wait_limit_ns = limit_ns;
-    if (launch_gemm<Elem, 0, 0, EPI_FWD_LSE>(tH, tW, tH /*no output box*/, g, s, num_sms) !=
+    if (launch_gemm2<Elem, 0, 0, EPI_FWD_LSE>(tH, tW, tH /*no output box*/, g, s, num_sms) !=
         cudaSuccess)
       return KD_ERR_CUDA;
     const int cblocks = cdiv(rows * 32, 256);
@@ -376,19 +488,19 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
   }
   CUtensorMap tW_k, tW_mn;
-  if (!make_map(&tW_k, W, F32, d, V, d, BK, BN)) return KD_ERR_CUDA;      // [V, d], K = d
+  if (!make_map(&tW_k, W, F32, d, V, d, BK, 128)) return KD_ERR_CUDA;     // [V, d], K = d
   if (!make_map(&tW_mn, W, F32, d, V, d, INNER, BK, true)) return KD_ERR_CUDA;  // K = V, N = d
-  CUtensorMap tDW_out;
+  CUtensorMap tDW_out, tHP_out;
   if (!make_out_map(&tDW_out, dW, true, d, V, d)) return KD_ERR_CUDA;
+  float* hpart = reinterpret_cast<float*>(w + L.hpart);
+  if (!make_out_map(&tHP_out, hpart, true, d, KD_DH_MAX_SPLIT * L.rows_pad, d)) return KD_ERR_CUDA;
   const float zscale = 1.4426950408889634f * inv_tau;
   const float inv_T_tau = static_cast<float>(1.0 / (static_cast<double>(T) * tau));
   for (int64_t c0 = 0; c0 < T; c0 += chunk) {
     const int64_t rows = (T - c0) < chunk ? (T - c0) : chunk;
     const Elem* hc = static_cast<const Elem*>(h) + c0 * d;
-    CUtensorMap tH_k, tH_mn, tDz_k, tDz_mn, tDz_out, tDH_out;
+    CUtensorMap tH_k, tH_mn, tDz_k, tDz_mn, tDz_out;
     if (!make_out_map(&tDz_out, dz, F32, V, rows, L.ldz)) return KD_ERR_CUDA;
-    if (!make_out_map(&tDH_out, static_cast<Elem*>(dH) + c0 * d, F32, d, rows, d))
-      return KD_ERR_CUDA;
     if (!make_map(&tH_k, hc, F32, d, rows, d, BK, BM)) return KD_ERR_CUDA;
     if (!make_map(&tH_mn, hc, F32, d, rows, d, INNER, BK, true)) return KD_ERR_CUDA;
     if (!make_map(&tDz_k, dz, F32, V, rows, L.ldz, BK, BM)) return KD_ERR_CUDA;
@@ -404,6 +516,7 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     g.n_tiles = cdiv(V, BN);
     g.k_blocks = cdiv(d, BK);
     g.m_fastest = 1;
+    g.k_split = 1;
     g.row0 = c0;
     g.V = V;
     g.Ktop = K;
@@ -418,7 +531,7 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     g.ldo = L.ldz;
     g.status = status;
     g.wait_limit_ns = limit_ns;
-    if (launch_gemm<Elem, 0, 0, EPI_BWD_DZ>(tH_k, tW_k, tDz_out, g, s, num_sms) != cudaSuccess)
+    if (launch_gemm2<Elem, 0, 0, EPI_BWD_DZ>(tH_k, tW_k, tDz_out, g, s, num_sms) != cudaSuccess)
       return KD_ERR_CUDA;
 
     // (2) dH_c = dz_c W : M = rows, N = d, K = V; A K-major, B MN-major
@@ -428,11 +541,28 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     gh.n_tiles = cdiv(d, BN);
     gh.k_blocks = cdiv(V, BK);
     gh.m_fastest = 1;
-    gh.out = dH;
+    gh.out = hpart;
     gh.ldo = d;
-    if (launch_gemm<Elem, 0, 1, EPI_STORE_H>(tDz_k, tW_mn, tDH_out, gh, s, num_sms) !=
+    gh.row0 = 0;
+    gh.split_rows = static_cast<int32_t>(L.rows_pad);
+    {
+      const int units1 = ((gh.M + BM2 - 1) / BM2) * gh.n_tiles;
+      gh.k_split = choose_dh_split(units1,
+                                   max_pair_clusters(gemm2_kernel<Elem, 0, 1, EPI_STORE_PARTIAL>,
+                                                     num_sms),
+                                   gh.k_blocks);
+    }
+    if (launch_gemm2<Elem, 0, 1, EPI_STORE_PARTIAL>(tDz_k, tW_mn, tHP_out, gh, s, num_sms) !=
         cudaSuccess)
       return KD_ERR_CUDA;
+    {
+      const int64_t n4 = rows * (d / 4);
+      dh_reduce_kernel<Elem><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(
+          hpart, gh.k_split, L.rows_pad, static_cast<int>(rows), d,
+          static_cast<Elem*>(dH) + c0 * d);
+      count_launch();
+      if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+    }
 
     // (3) dW (+)= dz_c^T h_c : M = V, N = d, K = rows; both operands MN-major
     GemmArgs gw = g;
@@ -447,7 +577,7 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     gw.out = dW;
     gw.ldo = d;
     gw.accumulate = (accumulate || c0 > 0) ? 1 : 0;
-    if (launch_gemm<Elem, 1, 1, EPI_ACCUM_W>(tDz_mn, tH_mn, tDW_out, gw, s, num_sms) !=
+    if (launch_gemm2<Elem, 1, 1, EPI_ACCUM_W>(tDz_mn, tH_mn, tDW_out, gw, s, num_sms) !=
         cudaSuccess)
       return KD_ERR_CUDA;
   }
