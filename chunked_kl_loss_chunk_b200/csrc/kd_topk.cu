@@ -30,6 +30,7 @@ constexpr int TK_SAMPLE = 4096;
 constexpr int TK_CAND_CAP = 2048;
 constexpr int TK_SEL_CAP = 1024;    // >= K
 constexpr int TK_UNROLL = 8;        // 16-byte loads in flight per thread
+constexpr int SAMPLE_PER_THREAD = TK_SAMPLE / TK_THREADS;   // 16
 
 // Order-preserving 16-bit key of a bf16 bit pattern: NaN -> 0 (lowest),
 // -0 -> key of +0, otherwise a monotone map of the value.
@@ -187,7 +188,68 @@ __device__ __forceinline__ void for_each_elem(const uint16_t* __restrict__ row, 
     f(row[i], static_cast<uint32_t>(i));
 }
 
-__global__ void __launch_bounds__(TK_THREADS)
+// Appends one element to the survivor buffer if it passes the threshold (the
+// exact per-element test; rarely reached from the streaming pass).
+__device__ __forceinline__ void offer(TopkSmem& sm, uint32_t bits, uint32_t i, float tf,
+                                     bool take_all) {
+  if (take_all || bf16_bits_to_float(bits) >= tf) {
+    const uint32_t pos = atomicAdd(&sm.n_cand, 1u);
+    if (pos < TK_CAND_CAP) sm.cand[pos] = composite(bf16_order_key(bits), i);
+  }
+}
+
+__device__ __noinline__ void offer8(TopkSmem& sm, uint4 q, uint32_t base, float tf,
+                                    bool take_all) {
+  const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    offer(sm, w[e] & 0xFFFFu, base + 2 * e, tf, take_all);
+    offer(sm, w[e] >> 16, base + 2 * e + 1, tf, take_all);
+  }
+}
+
+// Largest of the 8 bf16 values in q (NaNs ignored), as a float.
+__device__ __forceinline__ float max8_bf16(uint4 q) {
+  const __nv_bfloat162 a = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&q.x),
+                                   *reinterpret_cast<__nv_bfloat162*>(&q.y));
+  const __nv_bfloat162 b = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&q.z),
+                                   *reinterpret_cast<__nv_bfloat162*>(&q.w));
+  const __nv_bfloat162 c = __hmax2(a, b);
+  return fmaxf(__low2float(c), __high2float(c));
+}
+
+// The streaming pass: every element of the row meets the threshold once.  A
+// 16-byte vector is first screened by its maximum (three packed max ops and
+// one compare); only vectors that may hold a survivor take the exact path.
+__device__ __forceinline__ void stream_survivors(TopkSmem& sm, const uint16_t* __restrict__ row,
+                                                 int64_t V, float tf, bool take_all) {
+  const uintptr_t addr = reinterpret_cast<uintptr_t>(row);
+  int64_t head = ((16 - (addr & 15)) & 15) >> 1;
+  if (head > V) head = V;
+  for (int64_t i = threadIdx.x; i < head; i += TK_THREADS)
+    offer(sm, row[i], static_cast<uint32_t>(i), tf, take_all);
+  const int64_t nvec = (V - head) >> 3;
+  const uint4* vp = reinterpret_cast<const uint4*>(row + head);
+  for (int64_t j0 = threadIdx.x; j0 < nvec; j0 += TK_THREADS * TK_UNROLL) {
+    uint4 q[TK_UNROLL];
+#pragma unroll
+    for (int u = 0; u < TK_UNROLL; ++u) {
+      const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
+      q[u] = j < nvec ? __ldcs(vp + j) : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u,
+                                                   0xFF80FF80u);   // -inf: never passes
+    }
+#pragma unroll
+    for (int u = 0; u < TK_UNROLL; ++u) {
+      const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
+      if (j < nvec && (take_all || max8_bf16(q[u]) >= tf))
+        offer8(sm, q[u], static_cast<uint32_t>(head + (j << 3)), tf, take_all);
+    }
+  }
+  for (int64_t i = head + (nvec << 3) + threadIdx.x; i < V; i += TK_THREADS)
+    offer(sm, row[i], static_cast<uint32_t>(i), tf, take_all);
+}
+
+__global__ void __launch_bounds__(TK_THREADS, 4)
 topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int K,
                  float* __restrict__ out_vals, int32_t* __restrict__ out_idx) {
   extern __shared__ __align__(16) unsigned char tk_smem_raw[];
@@ -205,8 +267,39 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
     }
     __syncthreads();
     const int64_t S = V < TK_SAMPLE ? V : TK_SAMPLE;
-    for (int64_t i = tid; i < S; i += TK_THREADS)
-      atomicAdd(&sm.hist[bf16_order_key(row[i]) >> 4], 1u);
+    // The sample's keys stay in registers: SAMPLE_PER_THREAD per thread, loaded
+    // in one batch (16-byte vectors when the row is aligned and long enough).
+    uint32_t skey[SAMPLE_PER_THREAD];
+    if (S == TK_SAMPLE && (reinterpret_cast<uintptr_t>(row) & 15u) == 0) {
+      const uint4* vp = reinterpret_cast<const uint4*>(row);
+      uint4 q[SAMPLE_PER_THREAD / 8];
+#pragma unroll
+      for (int u = 0; u < SAMPLE_PER_THREAD / 8; ++u) q[u] = vp[tid + u * TK_THREADS];
+#pragma unroll
+      for (int u = 0; u < SAMPLE_PER_THREAD / 8; ++u) {
+        const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          skey[u * 8 + 2 * e] = bf16_order_key(w[e] & 0xFFFFu);
+          skey[u * 8 + 2 * e + 1] = bf16_order_key(w[e] >> 16);
+        }
+      }
+    } else {
+      uint32_t raw[SAMPLE_PER_THREAD];
+#pragma unroll
+      for (int u = 0; u < SAMPLE_PER_THREAD; ++u) {
+        const int64_t i = tid + static_cast<int64_t>(u) * TK_THREADS;
+        raw[u] = i < S ? row[i] : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < SAMPLE_PER_THREAD; ++u) {
+        const int64_t i = tid + static_cast<int64_t>(u) * TK_THREADS;
+        skey[u] = i < S ? bf16_order_key(raw[u]) : 0xFFFFFFFFu;   // marker: not sampled
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < SAMPLE_PER_THREAD; ++u)
+      if (skey[u] != 0xFFFFFFFFu) atomicAdd(&sm.hist[skey[u] >> 4], 1u);
     if (tid < 16) sm.hist16[tid] = 0u;
     __syncthreads();
     uint32_t target;
@@ -222,10 +315,9 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
     // Refine to the exact key of the target-th largest sample element: split
     // the threshold bin into its 16 keys.
     const uint32_t sb = sm.thr_bin, s_above = sm.thr_above;
-    for (int64_t i = tid; i < S; i += TK_THREADS) {
-      const uint32_t key = bf16_order_key(row[i]);
-      if ((key >> 4) == sb) atomicAdd(&sm.hist16[key & 15u], 1u);
-    }
+#pragma unroll
+    for (int u = 0; u < SAMPLE_PER_THREAD; ++u)
+      if (skey[u] != 0xFFFFFFFFu && (skey[u] >> 4) == sb) atomicAdd(&sm.hist16[skey[u] & 15u], 1u);
     __syncthreads();
     uint32_t L = sb << 4;                 // candidate iff order key >= L
     {
@@ -255,27 +347,66 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
     }
 
     // ---- 2. stream the row, keep survivors ------------------------------------
-    for_each_elem(row, V, [&](uint32_t bits, uint32_t i) {
-      const float x = bf16_bits_to_float(bits);
-      if (take_all || x >= tf) {
-        const uint32_t pos = atomicAdd(&sm.n_cand, 1u);
-        if (pos < TK_CAND_CAP) sm.cand[pos] = composite(bf16_order_key(bits), i);
-      }
-    });
+    stream_survivors(sm, row, V, tf, take_all);
     __syncthreads();
     const uint32_t n = sm.n_cand;
 
     if (n >= static_cast<uint32_t>(K) && n <= static_cast<uint32_t>(TK_CAND_CAP)) {
       // ---- 3. exact select among survivors -------------------------------------
-      const int np = next_pow2(static_cast<int>(n));
-      for (int i = static_cast<int>(n) + tid; i < np; i += TK_THREADS) sm.cand[i] = ~0ull;
+      // (a) the exact K-th largest key among the survivors (4096-bin histogram
+      //     of key >> 4, then the 16 keys of the threshold bin);
+      for (int b = tid; b < TK_BINS; b += TK_THREADS) sm.hist[b] = 0u;
+      if (tid < 16) sm.hist16[tid] = 0u;
       __syncthreads();
-      bitonic_sort(sm.cand, np);
-      for (int k = tid; k < K; k += TK_THREADS) {
-        const uint64_t c = sm.cand[k];
-        const uint32_t i = static_cast<uint32_t>(c);
-        out_idx[t * K + k] = static_cast<int32_t>(i);
-        out_vals[t * K + k] = bf16_bits_to_float(row[i]);
+      for (int i = tid; i < static_cast<int>(n); i += TK_THREADS)
+        atomicAdd(&sm.hist[(0xFFFFu - static_cast<uint32_t>(sm.cand[i] >> 32)) >> 4], 1u);
+      __syncthreads();
+      find_threshold_bin(sm, static_cast<uint32_t>(K));
+      const uint32_t cb = sm.thr_bin;
+      for (int i = tid; i < static_cast<int>(n); i += TK_THREADS) {
+        const uint32_t key = 0xFFFFu - static_cast<uint32_t>(sm.cand[i] >> 32);
+        if ((key >> 4) == cb) atomicAdd(&sm.hist16[key & 15u], 1u);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        uint32_t above = sm.thr_above, nib = 0, at = 0;
+        for (int j = 15; j >= 0; --j) {
+          if (above + sm.hist16[j] >= static_cast<uint32_t>(K)) {
+            nib = static_cast<uint32_t>(j);
+            at = sm.hist16[j];
+            break;
+          }
+          above += sm.hist16[j];
+        }
+        sm.thr_bin = (cb << 4) | nib;     // exact K-th key
+        sm.thr_above = above + at;        // survivors with key >= it
+        sm.n_sel = 0;
+      }
+      __syncthreads();
+      const uint32_t Tk = sm.thr_bin;
+      const bool compact = sm.thr_above <= static_cast<uint32_t>(TK_SEL_CAP);
+      // (b) keep the survivors with key >= Tk (the top K plus ties at Tk);
+      if (compact) {
+        for (int i = tid; i < static_cast<int>(n); i += TK_THREADS) {
+          const uint64_t c = sm.cand[i];
+          if (0xFFFFu - static_cast<uint32_t>(c >> 32) >= Tk) sm.sel[atomicAdd(&sm.n_sel, 1u)] = c;
+        }
+        __syncthreads();
+      }
+      // (c) rank: the composites are distinct (they contain the index), so an
+      //     entry's output position is the number of entries ordered before
+      //     it; those below K write themselves there, already in order.
+      const uint64_t* set = compact ? sm.sel : sm.cand;
+      const int ns = compact ? static_cast<int>(sm.n_sel) : static_cast<int>(n);
+      for (int i = tid; i < ns; i += TK_THREADS) {
+        const uint64_t c = set[i];
+        int rank = 0;
+        for (int j = 0; j < ns; ++j) rank += set[j] < c ? 1 : 0;
+        if (rank < K) {
+          const uint32_t idx = static_cast<uint32_t>(c);
+          out_idx[t * K + rank] = static_cast<int32_t>(idx);
+          out_vals[t * K + rank] = bf16_bits_to_float(row[idx]);
+        }
       }
       __syncthreads();
       continue;
