@@ -198,13 +198,24 @@ __device__ __forceinline__ void offer(TopkSmem& sm, uint32_t bits, uint32_t i, f
   }
 }
 
-__device__ __noinline__ void offer8(TopkSmem& sm, uint4 q, uint32_t base, float tf,
-                                    bool take_all) {
+// Exact test of the 8 elements of a screened vector: a pass mask built without
+// branches, then one append per passing element (usually one).
+__device__ __forceinline__ void offer8(TopkSmem& sm, uint4 q, uint32_t base, float tf,
+                                       bool take_all) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  uint32_t m = 0;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    offer(sm, w[e] & 0xFFFFu, base + 2 * e, tf, take_all);
-    offer(sm, w[e] >> 16, base + 2 * e + 1, tf, take_all);
+    m |= (__uint_as_float(w[e] << 16) >= tf ? 1u : 0u) << (2 * e);
+    m |= (__uint_as_float(w[e] & 0xFFFF0000u) >= tf ? 1u : 0u) << (2 * e + 1);
+  }
+  if (take_all) m = 0xFFu;
+  while (m) {
+    const int b = __ffs(m) - 1;
+    m &= m - 1;
+    const uint32_t bits = (w[b >> 1] >> ((b & 1) * 16)) & 0xFFFFu;
+    const uint32_t pos = atomicAdd(&sm.n_cand, 1u);
+    if (pos < TK_CAND_CAP) sm.cand[pos] = composite(bf16_order_key(bits), base + b);
   }
 }
 
