@@ -13,6 +13,10 @@ namespace kd {
 // the workspace).
 constexpr int KD_DH_MAX_SPLIT = 4;
 
+// Consecutive chunks whose dz the backward keeps side by side, so that dW is
+// updated once per group (its read-modify-write traffic falls by this factor).
+constexpr int KD_DW_GROUP = 2;
+
 // Byte offsets of the regions of a fused-loss workspace.
 struct WsLayout {
   size_t p_sorted = 0, idx_sorted = 0, stats = 0, kl = 0, scratch = 0, hpart = 0, total = 0;

@@ -381,7 +381,8 @@ WsLayout ws_layout(int64_t T, int64_t d, int64_t V, int K, int64_t chunk, int dt
   L.ldz = ((V + 63) / 64) * 64;
   const size_t n_tiles = static_cast<size_t>((V + BN - 1) / BN);
   const size_t part = static_cast<size_t>(rows) * n_tiles * 16;
-  const size_t dz = static_cast<size_t>(rows) * static_cast<size_t>(L.ldz) * es;
+  const size_t dz =
+      static_cast<size_t>(KD_DW_GROUP) * static_cast<size_t>(rows) * static_cast<size_t>(L.ldz) * es;
   L.scratch = off;
   off = al(off + (part > dz ? part : dz));
   L.rows_pad = ((rows + 255) / 256) * 256;
@@ -496,87 +497,104 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
   if (!make_out_map(&tHP_out, hpart, true, d, KD_DH_MAX_SPLIT * L.rows_pad, d)) return KD_ERR_CUDA;
   const float zscale = 1.4426950408889634f * inv_tau;
   const float inv_T_tau = static_cast<float>(1.0 / (static_cast<double>(T) * tau));
-  for (int64_t c0 = 0; c0 < T; c0 += chunk) {
-    const int64_t rows = (T - c0) < chunk ? (T - c0) : chunk;
-    const Elem* hc = static_cast<const Elem*>(h) + c0 * d;
-    CUtensorMap tH_k, tH_mn, tDz_k, tDz_mn, tDz_out;
-    if (!make_out_map(&tDz_out, dz, F32, V, rows, L.ldz)) return KD_ERR_CUDA;
-    if (!make_map(&tH_k, hc, F32, d, rows, d, BK, BM)) return KD_ERR_CUDA;
-    if (!make_map(&tH_mn, hc, F32, d, rows, d, INNER, BK, true)) return KD_ERR_CUDA;
-    if (!make_map(&tDz_k, dz, F32, V, rows, L.ldz, BK, BM)) return KD_ERR_CUDA;
-    if (!make_map(&tDz_mn, dz, F32, V, rows, L.ldz, INNER, BK, true)) return KD_ERR_CUDA;
+  // dz of KD_DW_GROUP consecutive chunks is kept side by side, so that dW is
+  // updated once per group with K = the group's rows (halving dW's
+  // read-modify-write traffic); dz and dH are formed chunk by chunk.
+  const int64_t group_rows = chunk * KD_DW_GROUP;
+  for (int64_t g0 = 0; g0 < T; g0 += group_rows) {
+    const int64_t grows = (T - g0) < group_rows ? (T - g0) : group_rows;
+    for (int64_t off = 0; off < grows; off += chunk) {
+      const int64_t c0 = g0 + off;
+      const int64_t rows = (grows - off) < chunk ? (grows - off) : chunk;
+      const Elem* hc = static_cast<const Elem*>(h) + c0 * d;
+      Elem* dzc = dz + off * L.ldz;                 // this chunk's rows of the group's dz
+      CUtensorMap tH_k, tDz_k, tDz_out;
+      if (!make_out_map(&tDz_out, dzc, F32, V, rows, L.ldz)) return KD_ERR_CUDA;
+      if (!make_map(&tH_k, hc, F32, d, rows, d, BK, BM)) return KD_ERR_CUDA;
+      if (!make_map(&tDz_k, dzc, F32, V, rows, L.ldz, BK, BM)) return KD_ERR_CUDA;
 
-    // (1) recompute z = h_c W^T; epilogue writes dz_c [rows, ldz]
-    GemmArgs g;
-    memset(&g, 0, sizeof(g));
-    g.M = static_cast<int32_t>(rows);
-    g.N = static_cast<int32_t>(V);
-    g.K = static_cast<int32_t>(d);
-    g.m_tiles = cdiv(rows, BM);
-    g.n_tiles = cdiv(V, BN);
-    g.k_blocks = cdiv(d, BK);
-    g.m_fastest = 1;
-    g.k_split = 1;
-    g.row0 = c0;
-    g.V = V;
-    g.Ktop = K;
-    g.zscale = zscale;
-    g.idx_sorted = idx_s;
-    g.p_sorted = p_s;
-    g.row_stats = stats;
-    g.lse = lse;
-    g.grad_loss = grad_loss;
-    g.inv_T_tau = inv_T_tau;
-    g.out = dz;
-    g.ldo = L.ldz;
-    g.status = status;
-    g.wait_limit_ns = limit_ns;
-    if (launch_gemm2<Elem, 0, 0, EPI_BWD_DZ>(tH_k, tW_k, tDz_out, g, s, num_sms) != cudaSuccess)
-      return KD_ERR_CUDA;
+      // (1) recompute z = h_c W^T; epilogue writes dz_c [rows, ldz]
+      GemmArgs g;
+      memset(&g, 0, sizeof(g));
+      g.M = static_cast<int32_t>(rows);
+      g.N = static_cast<int32_t>(V);
+      g.K = static_cast<int32_t>(d);
+      g.m_tiles = cdiv(rows, BM);
+      g.n_tiles = cdiv(V, BN);
+      g.k_blocks = cdiv(d, BK);
+      g.m_fastest = 1;
+      g.k_split = 1;
+      g.row0 = c0;
+      g.V = V;
+      g.Ktop = K;
+      g.zscale = zscale;
+      g.idx_sorted = idx_s;
+      g.p_sorted = p_s;
+      g.row_stats = stats;
+      g.lse = lse;
+      g.grad_loss = grad_loss;
+      g.inv_T_tau = inv_T_tau;
+      g.out = dzc;
+      g.ldo = L.ldz;
+      g.status = status;
+      g.wait_limit_ns = limit_ns;
+      if (launch_gemm2<Elem, 0, 0, EPI_BWD_DZ>(tH_k, tW_k, tDz_out, g, s, num_sms) != cudaSuccess)
+        return KD_ERR_CUDA;
 
-    // (2) dH_c = dz_c W : M = rows, N = d, K = V; A K-major, B MN-major
-    GemmArgs gh = g;
-    gh.N = static_cast<int32_t>(d);
-    gh.K = static_cast<int32_t>(V);
-    gh.n_tiles = cdiv(d, BN);
-    gh.k_blocks = cdiv(V, BK);
-    gh.m_fastest = 1;
-    gh.out = hpart;
-    gh.ldo = d;
-    gh.row0 = 0;
-    gh.split_rows = static_cast<int32_t>(L.rows_pad);
-    {
-      const int units1 = ((gh.M + BM2 - 1) / BM2) * gh.n_tiles;
-      gh.k_split = choose_dh_split(units1,
-                                   max_pair_clusters(gemm2_kernel<Elem, 0, 1, EPI_STORE_PARTIAL>,
-                                                     num_sms),
-                                   gh.k_blocks);
+      // (2) dH_c = dz_c W : M = rows, N = d, K = V; A K-major, B MN-major;
+      //     K split into even ranges whose fp32 partials are summed in order
+      GemmArgs gh = g;
+      gh.N = static_cast<int32_t>(d);
+      gh.K = static_cast<int32_t>(V);
+      gh.n_tiles = cdiv(d, BN);
+      gh.k_blocks = cdiv(V, BK);
+      gh.m_fastest = 1;
+      gh.out = hpart;
+      gh.ldo = d;
+      gh.row0 = 0;
+      gh.split_rows = static_cast<int32_t>(L.rows_pad);
+      {
+        const int units1 = ((gh.M + BM2 - 1) / BM2) * gh.n_tiles;
+        gh.k_split = choose_dh_split(units1,
+                                     max_pair_clusters(gemm2_kernel<Elem, 0, 1, EPI_STORE_PARTIAL>,
+                                                       num_sms),
+                                     gh.k_blocks);
+      }
+      if (launch_gemm2<Elem, 0, 1, EPI_STORE_PARTIAL>(tDz_k, tW_mn, tHP_out, gh, s, num_sms) !=
+          cudaSuccess)
+        return KD_ERR_CUDA;
+      {
+        const int64_t n4 = rows * (d / 4);
+        dh_reduce_kernel<Elem><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(
+            hpart, gh.k_split, L.rows_pad, static_cast<int>(rows), d,
+            static_cast<Elem*>(dH) + c0 * d);
+        count_launch();
+        if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+      }
     }
-    if (launch_gemm2<Elem, 0, 1, EPI_STORE_PARTIAL>(tDz_k, tW_mn, tHP_out, gh, s, num_sms) !=
-        cudaSuccess)
-      return KD_ERR_CUDA;
-    {
-      const int64_t n4 = rows * (d / 4);
-      dh_reduce_kernel<Elem><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(
-          hpart, gh.k_split, L.rows_pad, static_cast<int>(rows), d,
-          static_cast<Elem*>(dH) + c0 * d);
-      count_launch();
-      if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
-    }
 
-    // (3) dW (+)= dz_c^T h_c : M = V, N = d, K = rows; both operands MN-major
-    GemmArgs gw = g;
+    // (3) dW (+)= dz_g^T h_g over the group: M = V, N = d, K = grows; both
+    //     operands MN-major
+    const Elem* hg = static_cast<const Elem*>(h) + g0 * d;
+    CUtensorMap tH_mn, tDz_mn;
+    if (!make_map(&tH_mn, hg, F32, d, grows, d, INNER, BK, true)) return KD_ERR_CUDA;
+    if (!make_map(&tDz_mn, dz, F32, V, grows, L.ldz, INNER, BK, true)) return KD_ERR_CUDA;
+    GemmArgs gw;
+    memset(&gw, 0, sizeof(gw));
     gw.M = static_cast<int32_t>(V);
     gw.N = static_cast<int32_t>(d);
-    gw.K = static_cast<int32_t>(rows);
+    gw.K = static_cast<int32_t>(grows);
     gw.m_tiles = cdiv(V, BM);
     gw.n_tiles = cdiv(d, BN);
-    gw.k_blocks = cdiv(rows, BK);
+    gw.k_blocks = cdiv(grows, BK);
     gw.m_fastest = 0;              // tiles sharing one dz slab run together
-    gw.row0 = 0;
+    gw.k_split = 1;
+    gw.V = V;
     gw.out = dW;
     gw.ldo = d;
-    gw.accumulate = (accumulate || c0 > 0) ? 1 : 0;
+    gw.accumulate = (accumulate || g0 > 0) ? 1 : 0;
+    gw.status = status;
+    gw.wait_limit_ns = limit_ns;
     if (launch_gemm2<Elem, 1, 1, EPI_ACCUM_W>(tDz_mn, tH_mn, tDW_out, gw, s, num_sms) !=
         cudaSuccess)
       return KD_ERR_CUDA;

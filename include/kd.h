@@ -92,7 +92,11 @@ kd_status kd_topk_build(const void* logits, int dtype, int64_t T, int64_t V, int
 /* ------------------------------------------------------------------------ */
 
 /* Bytes of workspace kd_fused_kl_fwd / kd_fused_kl_bwd need for these sizes.
- * One workspace of this size serves both calls. */
+ * One workspace of this size serves both calls.  Besides O(T*K) for the
+ * prepared cache it holds, independent of T: the backward's dz of two
+ * consecutive chunks (2 * min(chunk,T) * V values of the operand dtype; dW is
+ * updated once per pair of chunks) and up to four fp32 K-split partials of one
+ * chunk's dH. */
 size_t kd_fused_kl_workspace_size(int64_t T, int64_t d, int64_t V, int K, int64_t chunk,
                                   int dtype);
 

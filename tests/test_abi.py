@@ -43,7 +43,7 @@ def test_workspace_sizes(lib):
     # fused: status + sorted cache (8 B/entry) + stats + kl + max(partials, dz)
     T, d, V, K, c = 32768, 4096, 131072, 100, 2048
     n = kd.kd_fused_kl_workspace_size(T, d, V, K, c, kd.KD_DTYPE_BF16)
-    dz = c * V * 2
+    dz = 2 * c * V * 2             # the backward keeps dz of two consecutive chunks
     cache = T * K * 8
     hpart = 4 * c * d * 4          # fp32 partials of up to 4 K-splits of dH
     assert dz + cache + hpart <= n <= dz + cache + hpart + T * 16 + 64 * 1024
