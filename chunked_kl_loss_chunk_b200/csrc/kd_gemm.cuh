@@ -1,41 +1,28 @@
-// kd_gemm.cuh -- persistent, warp-specialised tcgen05 GEMM for sm_100a with
-// the loss epilogues fused in.
+// kd_gemm.cuh -- what the tensor-core GEMM kernels of libkd share: tile
+// constants, per-dtype MMA parameters, launch arguments, and the loss
+// epilogues that drain an accumulator from TMEM.
 //
 //   D[m, n] = sum_k A[m, k] * B[n, k]          (fp32 accumulate in TMEM)
 //
-// One CTA per SM, 128x256 output tile, 128-byte-deep K stages fed by TMA with
-// 128-byte swizzle, 4 stages, two TMEM accumulators (2 x 256 columns) so the
-// epilogue of tile i overlaps the mainloop of tile i+1.
-//   warp 0      : TMA producer (one thread)
-//   warp 1      : TMEM allocator + MMA issuer (one thread)
-//   warps 2..5  : epilogue; warp w reads TMEM lanes 32*(w%4) .. +31, one
-//                 output row per thread, 32 columns per tcgen05.ld.
-// Operands may be K-major (rows of K contiguous) or MN-major (rows of M/N
-// contiguous); the UMMA descriptors and TMA boxes follow.
-//
-// Every wait is bounded (kd::mbar_wait); on a timeout or on an error recorded
-// by another CTA, each role leaves its loop, the producer waits for its own
-// copies in flight, the MMA thread for its own MMAs, and TMEM is freed.
+// Output tiles are 256 columns wide; each CTA owns 128 accumulator rows and
+// four epilogue warps, warp w reading TMEM lanes 32*(w%4) .. +31 (one output
+// row per thread, 32 columns per tcgen05.ld).  Operands may be K-major (rows
+// of K contiguous) or MN-major (rows of M/N contiguous).  The kernel itself is
+// in kd_gemm2.cuh.
 #pragma once
 
 #include "kd_common.cuh"
 
 namespace kd {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int STAGES = 4;
-constexpr int GEMM_THREADS = 192;
+constexpr int BM = 128;                        // accumulator rows per CTA
+constexpr int BN = 256;                        // output tile columns
+constexpr int GEMM_THREADS = 192;              // TMA warp, MMA warp, 4 epilogue warps
 constexpr int ROW_BYTES = 128;                 // K depth of a stage, in bytes
-constexpr int A_STAGE_BYTES = BM * ROW_BYTES;  // 16 KB
-constexpr int B_STAGE_BYTES = BN * ROW_BYTES;  // 32 KB
-constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
 constexpr int TMEM_COLS = 2 * BN;              // two accumulators
 constexpr int EPI_WARPS = 4;
 constexpr int EPI_BUF_BYTES = 32 * 128;        // one 32x32 fp32 (or 32x32 bf16) output box
 constexpr int EPI_SMEM_BYTES = EPI_WARPS * 2 * EPI_BUF_BYTES;   // double-buffered per warp
-constexpr int GEMM_SMEM_BYTES =
-    STAGES * STAGE_BYTES + EPI_SMEM_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
 template <typename Elem>
 struct ElemCfg;
@@ -268,195 +255,6 @@ __device__ __forceinline__ void run_epilogue(const GemmArgs& g, const CUtensorMa
       else stage_box_f32(box, lane, v);
       emit_box<Elem>(tmC, box, base, y_box, EPI == EPI_ACCUM_W && g.accumulate);
     }
-  }
-}
-
-// ----------------------------------------------------------------------------
-// The kernel.
-// ----------------------------------------------------------------------------
-template <typename Elem, int A_MN, int B_MN, int EPI>
-__global__ void __launch_bounds__(GEMM_THREADS, 1)
-gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-            const __grid_constant__ CUtensorMap tmC, const GemmArgs g) {
-  using C = ElemCfg<Elem>;
-  constexpr int BK = C::BK;
-  constexpr int INNER = ROW_BYTES / sizeof(Elem);        // MN elements per MN-major box
-  constexpr int BOX_BYTES = ROW_BYTES * BK;               // one MN-major box
-  constexpr uint32_t IDESC = umma_idesc(C::FMT, A_MN, B_MN, BM, BN);
-  constexpr int KSTEPS = BK / C::UMMA_K;                  // MMAs per stage (4)
-
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  unsigned char* sA = smem;
-  unsigned char* sB = smem + STAGES * A_STAGE_BYTES;
-  unsigned char* sEpi = smem + STAGES * STAGE_BYTES;      // [EPI_WARPS][2][EPI_BUF_BYTES]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + EPI_SMEM_BYTES);
-  uint64_t* full = bars;                 // [STAGES]
-  uint64_t* empty = bars + STAGES;       // [STAGES]
-  uint64_t* tfull = bars + 2 * STAGES;   // [2]
-  uint64_t* tempty = tfull + 2;          // [2]
-  uint64_t* drain = tempty + 2;          // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int num_tiles = g.m_tiles * g.n_tiles;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], 128);
-    }
-    mbar_init(drain, 1);
-    fence_mbar_init();
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-    if (EPI != EPI_FWD_LSE) tma_prefetch_desc(&tmC);
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t armed = 0;                 // bit s: stage s has been armed
-      uint32_t last_par = 0;              // bit s: parity of stage s's last arming
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const int mb = g.m_fastest ? tile % g.m_tiles : tile / g.n_tiles;
-        const int nb = g.m_fastest ? tile / g.m_tiles : tile % g.n_tiles;
-        for (int kb = 0; kb < g.k_blocks; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, g.wait_limit_ns, g.status)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          armed |= 1u << stage;
-          last_par = (last_par & ~(1u << stage)) | (phase << stage);
-          unsigned char* a = sA + stage * A_STAGE_BYTES;
-          unsigned char* b = sB + stage * B_STAGE_BYTES;
-          if (A_MN) {
-#pragma unroll
-            for (int j = 0; j < BM / INNER; ++j)
-              tma_load_2d(a + j * BOX_BYTES, &tmA, &full[stage], mb * BM + j * INNER, kb * BK);
-          } else {
-            tma_load_2d(a, &tmA, &full[stage], kb * BK, mb * BM);
-          }
-          if (B_MN) {
-#pragma unroll
-            for (int j = 0; j < BN / INNER; ++j)
-              tma_load_2d(b + j * BOX_BYTES, &tmB, &full[stage], nb * BN + j * INNER, kb * BK);
-          } else {
-            tma_load_2d(b, &tmB, &full[stage], kb * BK, nb * BN);
-          }
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      // Wait for every copy this thread started (no-op on the normal path).
-      for (int s = 0; s < STAGES; ++s)
-        if (armed & (1u << s)) mbar_drain(&full[s], (last_par >> s) & 1u, g.wait_limit_ns);
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, g.wait_limit_ns, g.status)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < g.k_blocks; ++kb) {
-          if (!mbar_wait(&full[stage], phase, g.wait_limit_ns, g.status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * A_STAGE_BYTES);
-          const uint32_t b0 = smem_u32(sB + stage * B_STAGE_BYTES);
-#pragma unroll
-          for (int k = 0; k < KSTEPS; ++k) {
-            // K-major: advance 32 bytes inside the swizzled row (SBO = 8 rows);
-            // MN-major: advance UMMA_K rows (LBO = next MN box, SBO = 8 rows).
-            const uint64_t ad =
-                A_MN ? umma_desc(a0 + k * C::UMMA_K * ROW_BYTES, BOX_BYTES, C::MN_SBO, C::MN_LAYOUT)
-                     : umma_desc(a0 + k * 32, 16, 1024, UMMA_LAYOUT_SW128);
-            const uint64_t bd =
-                B_MN ? umma_desc(b0 + k * C::UMMA_K * ROW_BYTES, BOX_BYTES, C::MN_SBO, C::MN_LAYOUT)
-                     : umma_desc(b0 + k * 32, 16, 1024, UMMA_LAYOUT_SW128);
-            const uint32_t accum = (kb | k) != 0 ? 1u : 0u;
-            if constexpr (C::FMT == 1) mma_f16(d_tmem, ad, bd, IDESC, accum);
-            else mma_tf32(d_tmem, ad, bd, IDESC, accum);
-          }
-          mma_commit(&empty[stage]);        // frees the stage once these MMAs finish
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (!ok) break;
-        mma_commit(&tfull[acc]);            // accumulator ready for the epilogue
-        if (++acc == 2) {
-          acc = 0;
-          acc_phase ^= 1u;
-        }
-      }
-      // Wait for every MMA this thread issued before TMEM is released.
-      mma_commit(drain);
-      mbar_drain(drain, 0, g.wait_limit_ns);
-    }
-    __syncwarp();
-  } else {
-    // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;                 // TMEM lane quadrant of this warp
-    unsigned char* boxes = sEpi + (warp - 2) * 2 * EPI_BUF_BYTES;
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int mb = g.m_fastest ? tile % g.m_tiles : tile / g.n_tiles;
-      const int nb = g.m_fastest ? tile / g.m_tiles : tile % g.n_tiles;
-      if (!mbar_wait(&tfull[acc], acc_phase, g.wait_limit_ns, g.status)) break;
-      tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                             static_cast<uint32_t>(acc * BN);
-      run_epilogue<Elem, EPI>(g, &tmC, mb * BM, nb, taddr, quad, lane, boxes);
-      __syncwarp();
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
-    }
-    // Every output box must have left shared memory and landed before exit.
-    if (lane == 0) bulk_wait<0>();
-    __syncwarp();
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 

@@ -343,23 +343,6 @@ int choose_dh_split(int units1, int nclusters, int k_blocks) {
   return best;
 }
 
-template <typename Elem, int A_MN, int B_MN, int EPI>
-cudaError_t launch_gemm(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc,
-                        GemmArgs g, cudaStream_t s, int num_sms) {
-  static constexpr int kKind[4] = {KD_GEMM_FWD_LSE, KD_GEMM_BWD_DZ, KD_GEMM_DH, KD_GEMM_DW};
-  auto kern = gemm_kernel<Elem, A_MN, B_MN, EPI>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       GEMM_SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  const int tiles = g.m_tiles * g.n_tiles;
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  profile_before(kKind[EPI], 2.0 * g.M * static_cast<double>(g.N) * g.K, s);
-  kern<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, s>>>(ta, tb, tc, g);
-  count_launch();
-  profile_after(s);
-  return cudaGetLastError();
-}
-
 inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
 }  // namespace
