@@ -229,6 +229,20 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ GPU arm
 
+def job_throughput(ms_local, tokens_per_rank, world, device):
+    """Whole-job throughput of independent replicas: the timed region is the
+    slowest rank's (max over ranks), the work is every rank's.  Returns
+    (ms of the slowest rank, tokens/s over all ranks)."""
+    ms = float(ms_local)
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms, tokens_per_rank * world / (ms / 1000.0)
+
+
 def run_kd(args, rank, world):
     import torch
     import torch.distributed as dist
@@ -318,15 +332,10 @@ def run_kd(args, rank, world):
     n_launch = kd.kd_launch_count() - n0
     clocks = sampler.stop() if sampler else None
     barrier()
-    ms_total = e0.elapsed_time(e1)
     peak_bytes = torch.cuda.max_memory_allocated(dev)
-    if world > 1:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total, value = job_throughput(e0.elapsed_time(e1), T * args.steps, world, dev)
     ms_step = ms_total / args.steps
     tokens = T * args.steps * world
-    value = tokens / (ms_total / 1000.0)
     flop_step = 8.0 * T * d * V
 
     # per-GEMM-kind breakdown from the live events
@@ -389,13 +398,9 @@ def run_kd(args, rank, world):
             consumed[i % 2].record(stream)
         b.record(stream)
         torch.cuda.synchronize()
-        ems = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([ems], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems, e2e_value = job_throughput(a.elapsed_time(b), T * args.steps, world, dev)
         assert bool(torch.isfinite(loss_host).all())
-        e2e = {"value": tokens / (ems / 1000.0), "unit": UNIT, "h2d_bytes_per_step": int(h2d),
+        e2e = {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": 4, "ms_per_step": ems / args.steps,
                "overlap": "inputs of step i+1 copied while step i computes (2 buffer sets)"}
         del sets
