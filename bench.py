@@ -409,7 +409,7 @@ def run_kd(args, rank, world):
         return
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, rows=args.cpu_rows or 16)
+        cpu = cpu_baseline(w, rows=args.cpu_rows or 128)
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -90,6 +90,8 @@ WORKLOADS = {
     # one and two 2048-position chunks of the 32K head: small cases for profiles
     "head-2k": dict(T=2048, d=4096, V=131072, K=100, chunk=2048, dtype="bf16"),
     "head-4k": dict(T=4096, d=4096, V=131072, K=100, chunk=2048, dtype="bf16"),
+    # two pairs of 2048-row chunks: the second dW launch adds into dW
+    "head-8k-c2048": dict(T=8192, d=4096, V=131072, K=100, chunk=2048, dtype="bf16"),
 }
 
 TOPK_WORKLOADS = {
