@@ -39,8 +39,13 @@ UNIT = "tokens/s"
 # gemm_topk_head-4k.md), valid only for the GEMM sources with this digest; the
 # roofline's "traffic" is null for any other source.
 NCU_TRAFFIC = {
-    "source_sha256_16": "e4030b4e36bf3456",
-    "per_launch_bytes": {"fwd_lse": 1.113e9, "bwd_dz": 1.628e9, "dH": 2.486e9, "dW": 4.66e9},
+    "source_sha256_16": "5c7479fc267328d5",
+    # dram__bytes_read.sum + dram__bytes_write.sum per launch of each GEMM kind,
+    # 2048-row chunks at d=4096, V=131072 (the launch shapes of the 32K head):
+    # fwd_lse from the 4K-position capture, the backward kinds from the
+    # 8K-position one; dW averages one storing and seven accumulating launches,
+    # the mix of a 32K step (16 chunks, dW once per pair of chunks)
+    "per_launch_bytes": {"fwd_lse": 1.138e9, "bwd_dz": 2.457e9, "dH": 3.985e9, "dW": 7.207e9},
 }
 
 
@@ -432,7 +437,7 @@ def run_kd(args, rank, world):
         "peak_mem_bytes": int(peak_bytes),
         "loss_path_bytes": int(loss_path_bytes),
         "dense_logits_grid_bytes_fp32": int(T * V * 4),
-        "roofline": {"bound": "tensor", "kernel": f"gemm_kernel ({dom[0]})",
+        "roofline": {"bound": "tensor", "kernel": f"gemm2_kernel ({dom[0]})",
                      "achieved": achieved, "peak": peak_sus, "unit": "TFLOP/s",
                      "frac": achieved / peak_sus,
                      "traffic": (NCU_TRAFFIC["per_launch_bytes"].get(dom[0])
@@ -463,12 +468,12 @@ def sweep_memory(args):
         h, W, vals, idx = inputs.make_loss_inputs(T, d, V, K, dtype=torch.bfloat16, seed=0, device=dev)
         torch.cuda.synchronize()
         torch.cuda.reset_peak_memory_stats(dev)
-        loss, lse, _, ws = kd.fused_kl_fwd(h, W, vals, idx, chunk, 1.0)
-        dH, dW, _ = kd.fused_kl_bwd(h, W, vals, idx, lse, chunk, 1.0, ws=ws)
+        loss, lse, kl, ws = kd.fused_kl_fwd(h, W, vals, idx, chunk, 1.0)
+        dH, dW, ws_b = kd.fused_kl_bwd(h, W, vals, idx, lse, chunk, 1.0, ws=ws)
         torch.cuda.synchronize()
         peak = torch.cuda.max_memory_allocated(dev) - base
         out.append({"T": T, "peak_bytes": int(peak), "dense_grid_fp32_bytes": T * V * 4})
-        del h, W, vals, idx, loss, lse, ws, dH, dW
+        del h, W, vals, idx, loss, lse, kl, ws, ws_b, dH, dW
     xs = [o["T"] for o in out]
     ys = [o["peak_bytes"] for o in out]
     n = len(xs)

@@ -244,12 +244,14 @@ def test_peak_memory_linear_in_T():
         h, W, vals, idx = inputs.make_loss_inputs(T, d, V, K, dtype=torch.bfloat16, seed=1, device=dev)
         torch.cuda.synchronize()
         torch.cuda.reset_peak_memory_stats(dev)        # the generator's temporaries are gone
-        loss, lse, _, ws = kd.fused_kl_fwd(h, W, vals, idx, chunk, 1.0)
-        dH, dW, _ = kd.fused_kl_bwd(h, W, vals, idx, lse, chunk, 1.0, ws=ws)
+        loss, lse, kl, ws = kd.fused_kl_fwd(h, W, vals, idx, chunk, 1.0)
+        dH, dW, ws_b = kd.fused_kl_bwd(h, W, vals, idx, lse, chunk, 1.0, ws=ws)
         torch.cuda.synchronize()
         assert kd.read_device_status(ws) == kd.KD_OK
         peaks.append(torch.cuda.max_memory_allocated(dev) - base)
-        del h, W, vals, idx, loss, lse, ws, dH, dW
+        # drop every reference (the workspace is returned twice), so that the
+        # next T's baseline holds none of this T's buffers
+        del h, W, vals, idx, loss, lse, kl, ws, ws_b, dH, dW
     x = np.array(Ts, np.float64)
     y = np.array(peaks, np.float64)
     b, a = np.polyfit(x, y, 1)
