@@ -27,6 +27,18 @@ What the pages fix, and the readings taken where they are silent:
   student logits, no tau^2 factor; the reduction is the mean over all T
   positions; 0 log 0 := 0.
 
+Two variants of the same objective (every function takes them as keywords):
+
+* ``cache="logprobs"``: the cache holds the teacher's log-probabilities from a
+  softmax over the FULL vocabulary, so the K cached entries carry only part of
+  the mass: p[t,k] = exp(vals[t,k]) as given (no renormalisation, no
+  temperature: it was applied when the teacher ran), S_t = sum_k p <= 1, and
+  sum p log p = sum_k p[t,k] vals[t,k].  The formulas above then hold with this
+  p and S unchanged (the gradient keeps its S_t softmax - p form).
+* ``tau_sq=True``: the loss and every gradient are multiplied by tau^2, the
+  usual temperature compensation of distillation; the per-row KL_t is returned
+  unscaled.
+
 All arithmetic is fp64.  Inputs are the exact values the GPU consumed (bf16 bit
 patterns are widened exactly).  Rows are processed in blocks only to bound host
 memory; every row's result is computed independently from its definition.
@@ -40,6 +52,7 @@ __all__ = [
     "bf16_bits_to_f64",
     "topk_rows",
     "teacher_distribution",
+    "loss_weight",
     "forward",
     "forward_rows",
     "backward",
@@ -103,12 +116,27 @@ def topk_rows(x, K: int):
 # a2: renormalised teacher distribution over the cached K entries
 # ---------------------------------------------------------------------------
 
-def teacher_distribution(vals, tau: float):
-    """p = softmax over the K cached teacher logits at temperature tau.
+CACHE_KINDS = ("logits", "logprobs")
+
+
+def teacher_distribution(vals, tau: float, cache: str = "logits"):
+    """Teacher probabilities at the K cached entries.
+
+    ``cache="logits"``: p = softmax over the K cached logits at temperature tau
+    (renormalised, S = 1).  ``cache="logprobs"``: p = exp(vals), the teacher's
+    own full-vocabulary probabilities, S <= 1.
 
     Returns (p [T,K], S [T] = sum_k p, plogp [T] = sum_k p log p with 0 log 0 = 0).
     """
-    b = _as_f64(vals) / tau
+    if cache not in CACHE_KINDS:
+        raise ValueError(f"cache must be one of {CACHE_KINDS}")
+    v = _as_f64(vals)
+    if cache == "logprobs":
+        p = np.exp(v)
+        S = p.sum(axis=1)
+        plogp = np.where(p > 0.0, p * np.where(p > 0.0, v, 0.0), 0.0).sum(axis=1)
+        return p, S, plogp
+    b = v / tau
     bmax = b.max(axis=1, keepdims=True)
     e = np.exp(b - bmax)
     p = e / e.sum(axis=1, keepdims=True)
@@ -116,6 +144,11 @@ def teacher_distribution(vals, tau: float):
     safe = np.where(p > 0.0, p, 1.0)
     plogp = np.where(p > 0.0, p * np.log(safe), 0.0).sum(axis=1)
     return p, S, plogp
+
+
+def loss_weight(tau: float, tau_sq: bool) -> float:
+    """Factor on the loss and its gradients: tau^2 with ``tau_sq``, else 1."""
+    return tau * tau if tau_sq else 1.0
 
 
 def _row_block_stats(h_rows, W, tau):
@@ -140,8 +173,10 @@ def _kl_from(a_rows, lse_rows, p_rows, idx_rows):
 # a3/a4: forward  (project, full-vocab logsumexp, gather at idx, fold, discard)
 # ---------------------------------------------------------------------------
 
-def forward(h, W, vals, idx, tau: float = 1.0, row_block: int = 256):
-    """Full forward: returns (loss, lse [T], kl [T]).
+def forward(h, W, vals, idx, tau: float = 1.0, row_block: int = 256, cache: str = "logits",
+            tau_sq: bool = False):
+    """Full forward: returns (loss, lse [T], kl [T]); loss carries the tau^2
+    factor when ``tau_sq``, kl does not.
 
     ``row_block`` only bounds host memory (each row is independent); results do
     not depend on it except through fp64 rounding of the final mean.
@@ -149,7 +184,7 @@ def forward(h, W, vals, idx, tau: float = 1.0, row_block: int = 256):
     h64, W64 = _as_f64(h), _as_f64(W)
     idx = np.asarray(idx)
     T = h64.shape[0]
-    p, _, _ = teacher_distribution(vals, tau)
+    p, _, _ = teacher_distribution(vals, tau, cache)
     lse = np.empty(T)
     kl = np.empty(T)
     for t0 in range(0, T, row_block):
@@ -157,14 +192,14 @@ def forward(h, W, vals, idx, tau: float = 1.0, row_block: int = 256):
         _, a, l = _row_block_stats(h64[t0:t1], W64, tau)
         lse[t0:t1] = l
         kl[t0:t1] = _kl_from(a, l, p[t0:t1], idx[t0:t1])
-    return kl.sum() / T, lse, kl
+    return loss_weight(tau, tau_sq) * (kl.sum() / T), lse, kl
 
 
-def forward_rows(h, W, vals, idx, tau: float, rows):
-    """lse and KL_t for a subset of rows (exact per row)."""
+def forward_rows(h, W, vals, idx, tau: float, rows, cache: str = "logits"):
+    """lse and KL_t (unscaled) for a subset of rows (exact per row)."""
     rows = np.asarray(rows)
     h64 = _as_f64(np.asarray(h)[rows])
-    p, _, _ = teacher_distribution(np.asarray(vals)[rows], tau)
+    p, _, _ = teacher_distribution(np.asarray(vals)[rows], tau, cache)
     _, a, l = _row_block_stats(h64, _as_f64(W), tau)
     return l, _kl_from(a, l, p, np.asarray(idx)[rows])
 
@@ -181,13 +216,14 @@ def _dz_block(a, lse, p, S, idx, scale):
     return dz * scale
 
 
-def backward(h, W, vals, idx, tau: float = 1.0, g: float = 1.0, row_block: int = 256):
+def backward(h, W, vals, idx, tau: float = 1.0, g: float = 1.0, row_block: int = 256,
+             cache: str = "logits", tau_sq: bool = False):
     """Full backward: returns (dH [T,d], dW [V,d]) in fp64."""
     h64, W64 = _as_f64(h), _as_f64(W)
     idx = np.asarray(idx)
     T = h64.shape[0]
-    p, S, _ = teacher_distribution(vals, tau)
-    scale = g / (T * tau)
+    p, S, _ = teacher_distribution(vals, tau, cache)
+    scale = loss_weight(tau, tau_sq) * g / (T * tau)
     dH = np.empty_like(h64)
     dW = np.zeros_like(W64)
     for t0 in range(0, T, row_block):
@@ -199,19 +235,22 @@ def backward(h, W, vals, idx, tau: float = 1.0, g: float = 1.0, row_block: int =
     return dH, dW
 
 
-def backward_dH_rows(h, W, vals, idx, tau: float, rows, T_total: int, g: float = 1.0):
+def backward_dH_rows(h, W, vals, idx, tau: float, rows, T_total: int, g: float = 1.0,
+                     cache: str = "logits", tau_sq: bool = False):
     """dH for a subset of rows; each row needs only its own LSE."""
     rows = np.asarray(rows)
     h64 = _as_f64(np.asarray(h)[rows])
     W64 = _as_f64(W)
-    p, S, _ = teacher_distribution(np.asarray(vals)[rows], tau)
+    p, S, _ = teacher_distribution(np.asarray(vals)[rows], tau, cache)
     _, a, l = _row_block_stats(h64, W64, tau)
-    dz = _dz_block(a, l, p, S, np.asarray(idx)[rows], g / (T_total * tau))
+    dz = _dz_block(a, l, p, S, np.asarray(idx)[rows],
+                   loss_weight(tau, tau_sq) * g / (T_total * tau))
     return dz @ W64
 
 
 def backward_dW_rows(h, W, vals, idx, tau: float, vrows, g: float = 1.0,
-                     lse=None, row_block: int = 256):
+                     lse=None, row_block: int = 256, cache: str = "logits",
+                     tau_sq: bool = False):
     """dW[v,:] for a subset of vocabulary rows v.
 
     Needs LSE_t of every position (one full fp64 projection) unless the
@@ -227,13 +266,13 @@ def backward_dW_rows(h, W, vals, idx, tau: float, vrows, g: float = 1.0,
         for t0 in range(0, T, row_block):
             t1 = min(T, t0 + row_block)
             lse[t0:t1] = _row_block_stats(h64[t0:t1], W64, tau)[2]
-    p, S, _ = teacher_distribution(vals, tau)
+    p, S, _ = teacher_distribution(vals, tau, cache)
     a_sel = (h64 @ W64[vrows].T) / tau                       # [T, |vrows|]
     dz = S[:, None] * np.exp(a_sel - lse[:, None])           # softmax part
     for j, v in enumerate(vrows):
         hit = idx == v                                        # [T, K]
         dz[:, j] -= (p * hit).sum(axis=1)                     # scatter part
-    dz *= g / (T * tau)
+    dz *= loss_weight(tau, tau_sq) * g / (T * tau)
     return dz.T @ h64                                         # [|vrows|, d]
 
 
@@ -241,7 +280,8 @@ def backward_dW_rows(h, W, vals, idx, tau: float, vrows, g: float = 1.0,
 # Dense brute force: the [T, V] grid the fused method avoids
 # ---------------------------------------------------------------------------
 
-def dense_bruteforce_loss(h, W, vals, idx, tau: float = 1.0):
+def dense_bruteforce_loss(h, W, vals, idx, tau: float = 1.0, cache: str = "logits",
+                          tau_sq: bool = False):
     """Materialise full student log-probs and a dense scattered teacher
     distribution over [T, V] and sum p (log p - log q) over its support.
     Only for tiny shapes ([DD] "The two changes" describes this grid as what a
@@ -254,7 +294,10 @@ def dense_bruteforce_loss(h, W, vals, idx, tau: float = 1.0):
     idx = np.asarray(idx).astype(np.int64)
     T, V = h64.shape[0], W64.shape[0]
     logq = log_softmax((h64 @ W64.T) / tau, axis=1)          # [T, V]
-    pt = softmax(_as_f64(vals) / tau, axis=1)                 # [T, K]
+    if cache == "logprobs":
+        pt = np.exp(_as_f64(vals))                            # teacher's own probabilities
+    else:
+        pt = softmax(_as_f64(vals) / tau, axis=1)             # [T, K]
     P = np.zeros((T, V))
     for t in range(T):
         for k in range(idx.shape[1]):
@@ -263,4 +306,4 @@ def dense_bruteforce_loss(h, W, vals, idx, tau: float = 1.0):
     for t in range(T):
         sup = P[t] > 0
         total += float((P[t, sup] * (np.log(P[t, sup]) - logq[t, sup])).sum())
-    return total / T
+    return (tau * tau if tau_sq else 1.0) * total / T

@@ -243,6 +243,168 @@ def test_backward_chunk_invariance():
         assert np.allclose(dH, ref[0], atol=1e-15) and np.allclose(dW, ref[1], atol=1e-14)
 
 
+# ---------------------------------------------------------------- variants:
+# a cache of full-vocabulary teacher log-probabilities (S = sum p < 1), and the
+# tau^2 factor on loss and gradients
+
+def _logprob_cache(T, K, seed=5, mass=(0.3, 0.95)):
+    """Unnormalised teacher log-probs: K entries of a distribution whose other
+    entries (the tail the cache dropped) hold 1 - S of the mass."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((T, K)) * math.sqrt(2.0)
+    S = rng.uniform(*mass, size=T)
+    lp = torch.log_softmax(torch.tensor(x), dim=1).numpy() + np.log(S)[:, None]
+    return lp, S
+
+
+def test_logprob_cache_hand_example():
+    """V = 2, d = 1, W = [ln 3, 0], h = 1: z = (ln 3, 0), q = (3/4, 1/4),
+    LSE = ln 4.  One cached entry, token 0 with p = 1/2 (S = 1/2):
+    KL = (1/2)(ln 1/2 - ln 3/4) = (1/2) ln 2/3;  dz = S q - p~ = (-1/8, 1/8);
+    dH = dz W = -(ln 3)/8;  dW = dz^T h = (-1/8, 1/8).
+    With tau = 2 and the tau^2 factor: q0 = sqrt3/(1 + sqrt3) = (3 - sqrt3)/2,
+    loss = 4 (1/2)(ln 1/2 - ln q0), dz = 4/(1*2) (S q - p~) = (q0 - 1, 1 - q0)."""
+    h = np.array([[1.0]])
+    W = np.array([[math.log(3.0)], [0.0]])
+    vals = np.array([[math.log(0.5)]])
+    idx = np.array([[0]], np.int32)
+    loss, lse, kl = oracle.forward(h, W, vals, idx, 1.0, cache="logprobs")
+    assert abs(loss - 0.5 * math.log(2.0 / 3.0)) < 1e-15
+    assert abs(lse[0] - math.log(4.0)) < 1e-15
+    dH, dW = oracle.backward(h, W, vals, idx, 1.0, cache="logprobs")
+    assert abs(dH[0, 0] + math.log(3.0) / 8) < 1e-15
+    assert np.allclose(dW[:, 0], [-0.125, 0.125], atol=1e-16)
+
+    q0 = (3.0 - math.sqrt(3.0)) / 2.0
+    loss2, lse2, kl2 = oracle.forward(h, W, vals, idx, 2.0, cache="logprobs", tau_sq=True)
+    assert abs(loss2 - 4 * 0.5 * (math.log(0.5) - math.log(q0))) < 1e-14
+    assert abs(kl2[0] - 0.5 * (math.log(0.5) - math.log(q0))) < 1e-15     # kl unscaled
+    assert abs(lse2[0] - math.log(math.sqrt(3.0) + 1.0)) < 1e-15
+    dH2, dW2 = oracle.backward(h, W, vals, idx, 2.0, cache="logprobs", tau_sq=True)
+    assert np.allclose(dW2[:, 0], [q0 - 1.0, 1.0 - q0], atol=1e-15)
+    assert abs(dH2[0, 0] - (q0 - 1.0) * math.log(3.0)) < 1e-15
+
+
+def test_logprob_uniform_student_closed_form():
+    """W = 0 -> q = 1/V -> KL_t = sum_k p log p + S ln V with p = exp(vals)."""
+    T, d, V, K = 9, 6, 23, 5
+    h, W, _, idx = _tiny(T=T, d=d, V=V, K=K)
+    lp, S = _logprob_cache(T, K)
+    for tau in (1.0, 0.7):
+        loss, lse, kl = oracle.forward(h, np.zeros_like(W), lp, idx, tau, cache="logprobs")
+        p = np.exp(lp)
+        assert np.allclose(p.sum(axis=1), S, atol=1e-14)
+        p2, S2, plogp2 = oracle.teacher_distribution(lp, tau, cache="logprobs")
+        assert np.allclose(S2, S, atol=1e-14) and np.allclose(plogp2, (p * lp).sum(axis=1), atol=1e-14)
+        assert np.allclose(kl, (p * lp).sum(axis=1) + S * math.log(V), atol=1e-13)
+        assert np.all(kl < (p * lp).sum(axis=1) + math.log(V))  # S < 1 lowers the loss
+
+
+def test_logprob_full_vocab_is_full_kl():
+    """K = V, vals = the teacher's log-softmax -> the full KL of torch's kl_div."""
+    T, d, V = 7, 5, 11
+    h, W, tl, idx = _tiny(T=T, d=d, V=V, K=V)
+    lp = torch.log_softmax(torch.tensor(tl), dim=1).numpy()
+    for tau in (1.0, 1.7):
+        loss, _, _ = oracle.forward(h, W, lp, idx, tau, cache="logprobs")
+        logq = torch.log_softmax(torch.tensor(h @ W.T / tau), dim=1)
+        # teacher log-probs in vocabulary order
+        lpv = np.zeros((T, V))
+        for t in range(T):
+            lpv[t, idx[t]] = lp[t]
+        ref = torch.nn.functional.kl_div(logq, torch.tensor(lpv), reduction="sum",
+                                         log_target=True).item() / T
+        assert abs(loss - ref) < 1e-12
+
+
+def test_logprob_cache_of_renormalised_teacher_equals_logits_cache():
+    """vals' = log softmax_K(vals / tau) read as log-probs gives the logits
+    cache's loss and gradients at the same tau."""
+    h, W, vals, idx = _tiny(T=8, d=5, V=19, K=4)
+    for tau in (1.0, 0.8):
+        lp = torch.log_softmax(torch.tensor(vals / tau), dim=1).numpy()
+        a = oracle.forward(h, W, vals, idx, tau)
+        b = oracle.forward(h, W, lp, idx, tau, cache="logprobs")
+        assert abs(a[0] - b[0]) < 1e-14 and np.allclose(a[2], b[2], atol=1e-14)
+        ga = oracle.backward(h, W, vals, idx, tau, 1.3)
+        gb = oracle.backward(h, W, lp, idx, tau, 1.3, cache="logprobs")
+        assert np.allclose(ga[0], gb[0], atol=1e-15) and np.allclose(ga[1], gb[1], atol=1e-15)
+
+
+def test_logprob_dense_bruteforce():
+    T, d, V, K = 13, 7, 29, 6
+    h, W, _, idx = _tiny(T=T, d=d, V=V, K=K)
+    lp, _ = _logprob_cache(T, K, seed=2)
+    for tau, sq in ((1.0, False), (0.5, True), (2.0, True)):
+        dense = oracle.dense_bruteforce_loss(h, W, lp, idx, tau, cache="logprobs", tau_sq=sq)
+        loss, _, kl = oracle.forward(h, W, lp, idx, tau, cache="logprobs", tau_sq=sq)
+        assert abs(loss - dense) < 1e-12
+
+
+def _fd_check_variant(tau, g, cache, tau_sq):
+    T, d, V, K = 5, 4, 13, 4
+    h, W, vals, idx = _tiny(T=T, d=d, V=V, K=K, seed=11)
+    if cache == "logprobs":
+        vals, _ = _logprob_cache(T, K, seed=4)
+    kw = dict(cache=cache, tau_sq=tau_sq)
+    dH, dW = oracle.backward(h, W, vals, idx, tau, g, **kw)
+    rng = np.random.default_rng(7)
+    eps = 1e-6
+    f = lambda hh, WW: oracle.forward(hh, WW, vals, idx, tau, **kw)[0]
+    for _ in range(20):
+        t, j = rng.integers(T), rng.integers(d)
+        hp, hm = h.copy(), h.copy()
+        hp[t, j] += eps
+        hm[t, j] -= eps
+        fd = g * (f(hp, W) - f(hm, W)) / (2 * eps)
+        assert abs(fd - dH[t, j]) <= 1e-6 * max(1.0, abs(dH[t, j])) + 1e-9
+        v, j = rng.integers(V), rng.integers(d)
+        Wp, Wm = W.copy(), W.copy()
+        Wp[v, j] += eps
+        Wm[v, j] -= eps
+        fd = g * (f(h, Wp) - f(h, Wm)) / (2 * eps)
+        assert abs(fd - dW[v, j]) <= 1e-6 * max(1.0, abs(dW[v, j])) + 1e-9
+
+
+def test_variant_gradients_finite_differences():
+    _fd_check_variant(1.0, 1.0, "logprobs", False)
+    _fd_check_variant(0.6, 2.5, "logprobs", True)
+    _fd_check_variant(1.7, 0.5, "logits", True)
+
+
+def test_tau_sq_high_temperature_limit_is_logit_matching():
+    """With a dense teacher (K = V) and the tau^2 factor, as tau grows the loss
+    tends to (1/(2 V T)) sum_t |w_t - u_t|^2 and dz to g (w - u)/(T V), where u, w
+    are the teacher's and the student's logits with their row means removed
+    (the high-temperature limit of distillation).  Both errors shrink as 1/tau."""
+    T, d, V = 6, 5, 11
+    h, W, x, idx = _tiny(T=T, d=d, V=V, K=V, seed=9)
+    z = h @ W.T
+    xv = np.zeros((T, V))
+    for t in range(T):
+        xv[t, idx[t]] = x[t]
+    u = xv - xv.mean(axis=1, keepdims=True)
+    w = z - z.mean(axis=1, keepdims=True)
+    lim_loss = ((w - u) ** 2).sum() / (2 * V * T)
+    lim_dW = ((w - u) / (T * V)).T @ h
+    errs = []
+    for tau in (1e2, 1e3):
+        loss, _, _ = oracle.forward(h, W, x, idx, tau, tau_sq=True)
+        _, dW = oracle.backward(h, W, x, idx, tau, tau_sq=True)
+        errs.append((abs(loss - lim_loss) / lim_loss,
+                     np.abs(dW - lim_dW).max() / np.abs(lim_dW).max()))
+    assert errs[1][0] < 2e-3 and errs[1][1] < 2e-3
+    assert errs[1][0] < 0.2 * errs[0][0] and errs[1][1] < 0.2 * errs[0][1]
+    # without the factor the loss vanishes as 1/tau^2
+    plain, _, _ = oracle.forward(h, W, x, idx, 1e3)
+    assert abs(plain * 1e6 - lim_loss) / lim_loss < 2e-3
+
+
+def test_unknown_cache_kind_rejected():
+    with pytest.raises(ValueError):
+        oracle.teacher_distribution(np.zeros((1, 2)), 1.0, cache="probs")
+
+
 # ---------------------------------------------------------------- inputs
 
 def test_input_generator_shapes_and_distinct_indices():
