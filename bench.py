@@ -36,16 +36,15 @@ UNIT = "tokens/s"
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
 # ncu capture of launches shaped exactly like the bench's (profiles/
-# gemm_topk_head-4k.md), valid only for the GEMM sources with this digest; the
-# roofline's "traffic" is null for any other source.
+# gemm2_step_head-8k-c2048.md), valid only for the GEMM sources with this
+# digest; the roofline's "traffic" is null for any other source.
 NCU_TRAFFIC = {
-    "source_sha256_16": "5c7479fc267328d5",
+    "source_sha256_16": "216e20f713104a8f",
     # dram__bytes_read.sum + dram__bytes_write.sum per launch of each GEMM kind,
-    # 2048-row chunks at d=4096, V=131072 (the launch shapes of the 32K head):
-    # fwd_lse from the 4K-position capture, the backward kinds from the
-    # 8K-position one; dW averages one storing and seven accumulating launches,
-    # the mix of a 32K step (16 chunks, dW once per pair of chunks)
-    "per_launch_bytes": {"fwd_lse": 1.138e9, "bwd_dz": 2.457e9, "dH": 3.985e9, "dW": 7.207e9},
+    # from one capture of all 14 GEMM launches of a head-8k-c2048 step (2048-row
+    # chunks at d=4096, V=131072: the launch shapes of the 32K head); dW is the
+    # mix of a 32K step, one storing and seven accumulating launches
+    "per_launch_bytes": {"fwd_lse": 1.199e9, "bwd_dz": 1.830e9, "dH": 3.295e9, "dW": 6.027e9},
 }
 
 
@@ -279,6 +278,7 @@ def run_kd(args, rank, world):
     code = kd.KD_DTYPE_BF16 if dt == torch.bfloat16 else kd.KD_DTYPE_F32
     ev_topk = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     ev_fwd = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev_bwd = torch.cuda.Event(enable_timing=True)
 
     def step(timing=None, inp=None):
         hh, WW, xx = inp if inp is not None else (h, W, logits)
@@ -299,9 +299,11 @@ def run_kd(args, rank, world):
         if st != 0:
             raise RuntimeError(f"libkd call failed ({st})")
         if timing is not None:
+            ev_bwd.record()
             torch.cuda.synchronize()
             timing["topk_ms"].append(ev_topk[0].elapsed_time(ev_topk[1]))
             timing["fwd_ms"].append(ev_topk[1].elapsed_time(ev_fwd[1]))
+            timing["bwd_ms"].append(ev_fwd[1].elapsed_time(ev_bwd))
 
     def barrier():
         if world > 1:
@@ -313,9 +315,9 @@ def run_kd(args, rank, world):
     torch.cuda.synchronize()
     assert kd.read_device_status(ws) == kd.KD_OK
 
-    # component timings (separate, untimed-region passes)
-    comp = {"topk_ms": [], "fwd_ms": []}
-    for _ in range(2):
+    # component timings (separate passes outside the timed region; medians)
+    comp = {"topk_ms": [], "fwd_ms": [], "bwd_ms": []}
+    for _ in range(5):
         step(comp)
 
     prof = kd.GemmProfiler(capacity=4 * ((T + chunk - 1) // chunk) * args.steps + 16)
@@ -358,6 +360,7 @@ def run_kd(args, rank, world):
     gemm_ms_step = sum(v["ms"] for v in kinds.values()) / args.steps
     topk_ms = statistics.median(comp["topk_ms"])
     fwd_ms = statistics.median(comp["fwd_ms"])
+    bwd_ms = statistics.median(comp["bwd_ms"])
     loss_ms = ms_step - topk_ms
     loss_tflops = flop_step / (loss_ms / 1000.0) / 1e12
 
@@ -426,7 +429,7 @@ def run_kd(args, rank, world):
                           "tflops": loss_tflops,
                           "frac_bf16_peak_sustained": loss_tflops / peak_sus,
                           "frac_bf16_peak_burst": loss_tflops / float(peaks["bf16_tflops"]),
-                          "fwd_ms": fwd_ms, "bwd_ms": loss_ms - fwd_ms,
+                          "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
                           "gemm_ms": gemm_ms_step},
         "topk_build": {"ms": topk_ms, "gbs": (T * V * 2 + T * K * 8) / (topk_ms / 1000.0) / 1e9,
                        "frac_hbm_peak": (T * V * 2 + T * K * 8) / (topk_ms / 1000.0) / 1e9

@@ -28,12 +28,12 @@ WsLayout ws_layout(int64_t T, int64_t d, int64_t V, int K, int64_t chunk, int dt
 
 kd_status fused_fwd(const void* h, const void* W, int dtype, int64_t T, int64_t d, int64_t V,
                     const float* t_vals, const int32_t* t_idx, int K, int64_t chunk, float tau,
-                    float* loss, float* lse, float* kl_rows, void* ws, cudaStream_t s,
+                    uint32_t flags, float* loss, float* lse, float* kl_rows, void* ws, cudaStream_t s,
                     int num_sms, uint64_t limit_ns);
 
 kd_status fused_bwd(const void* h, const void* W, int dtype, int64_t T, int64_t d, int64_t V,
                     const float* t_vals, const int32_t* t_idx, int K, int64_t chunk, float tau,
-                    const float* lse, const float* grad_loss, void* dH, float* dW,
+                    uint32_t flags, const float* lse, const float* grad_loss, void* dH, float* dW,
                     int accumulate, void* ws, cudaStream_t s, int num_sms, uint64_t limit_ns);
 
 cudaError_t launch_topk_bf16(const void* logits, int64_t T, int64_t V, int K, float* out_vals,

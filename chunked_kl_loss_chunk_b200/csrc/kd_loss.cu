@@ -17,18 +17,26 @@
 
 namespace kd {
 
+// Factor on the loss and on every gradient: tau^2 under KD_KL_TAU_SQUARED
+// (the usual temperature compensation of distillation), else 1.
+static inline double loss_weight(float tau, uint32_t flags) {
+  return (flags & KD_KL_TAU_SQUARED) ? static_cast<double>(tau) * tau : 1.0;
+}
+
 // ----------------------------------------------------------------------------
 // K2: cache prep.  One warp per position: p = softmax(vals / tau) over the K
-// cached logits, S = sum p, sum p log p, then the (index, p) pairs sorted by
-// index ascending.  Indices outside [0, V) or repeated in a row record
-// KD_ERR_BAD_INDEX; such entries get p = 0 and are moved past V.
+// cached logits (or, for a cache of full-vocabulary log-probabilities,
+// p = exp(vals) with no renormalisation), S = sum p, sum p log p, then the
+// (index, p) pairs sorted by index ascending.  Indices outside [0, V) or
+// repeated in a row record KD_ERR_BAD_INDEX; such entries get p = 0 and are
+// moved past V.
 // ----------------------------------------------------------------------------
 constexpr int PREP_WARPS = 4;
 constexpr int PREP_MAXK = 1024;
 
 __global__ void __launch_bounds__(PREP_WARPS * 32)
 prep_kernel(const float* __restrict__ vals, const int32_t* __restrict__ idx, int64_t T, int K,
-            int64_t V, float inv_tau, int32_t* __restrict__ idx_sorted,
+            int64_t V, float inv_tau, int logprob, int32_t* __restrict__ idx_sorted,
             float* __restrict__ p_sorted, float2* __restrict__ stats, uint32_t* status) {
   extern __shared__ __align__(16) unsigned char prep_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -40,19 +48,25 @@ prep_kernel(const float* __restrict__ vals, const int32_t* __restrict__ idx, int
        t += static_cast<int64_t>(gridDim.x) * PREP_WARPS) {
     const float* vr = vals + t * K;
     const int32_t* ir = idx + t * K;
-    float mx = -INFINITY;
-    for (int k = lane; k < K; k += 32) mx = fmaxf(mx, vr[k] * inv_tau);
+    // cached logits: p = softmax over the K entries at temperature tau;
+    // cached log-probabilities: p = exp(vals) as given (S <= 1).
+    float mx = 0.f, inv_se = 1.f;
+    if (!logprob) {
+      mx = -INFINITY;
+      for (int k = lane; k < K; k += 32) mx = fmaxf(mx, vr[k] * inv_tau);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    float se = 0.f;
-    for (int k = lane; k < K; k += 32) se += expf(vr[k] * inv_tau - mx);
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float se = 0.f;
+      for (int k = lane; k < K; k += 32) se += expf(vr[k] * inv_tau - mx);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
-    const float inv_se = 1.f / se;
+      for (int o = 16; o > 0; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
+      inv_se = 1.f / se;
+    }
     float S = 0.f, plogp = 0.f;
     bool bad = false;
     for (int k = lane; k < K; k += 32) {
-      float p = expf(vr[k] * inv_tau - mx) * inv_se;
+      const float b = logprob ? vr[k] : vr[k] * inv_tau - mx;
+      float p = expf(b) * inv_se;
       int32_t i = ir[k];
       if (i < 0 || static_cast<int64_t>(i) >= V) {
         bad = true;
@@ -60,7 +74,7 @@ prep_kernel(const float* __restrict__ vals, const int32_t* __restrict__ idx, int
         i = INT32_MAX;
       }
       S += p;
-      if (p > 0.f) plogp += p * logf(p);
+      if (p > 0.f) plogp += p * (logprob ? b : logf(p));
       buf[k] = (static_cast<uint64_t>(static_cast<uint32_t>(i)) << 32) | __float_as_uint(p);
     }
     for (int k = K + lane; k < np; k += 32) buf[k] = ~0ull;
@@ -186,7 +200,7 @@ dh_reduce_kernel(const float* __restrict__ part, int k_split, int64_t split_rows
 // Deterministic mean of kl[0..T): one block, fixed per-thread strides, fixed
 // tree; fp64 accumulation.
 __global__ void __launch_bounds__(1024)
-mean_kernel(const float* __restrict__ kl, int64_t T, float* __restrict__ loss) {
+mean_kernel(const float* __restrict__ kl, int64_t T, double scale, float* __restrict__ loss) {
   __shared__ double part[1024];
   double acc = 0.0;
   for (int64_t i = threadIdx.x; i < T; i += 1024) acc += static_cast<double>(kl[i]);
@@ -196,7 +210,7 @@ mean_kernel(const float* __restrict__ kl, int64_t T, float* __restrict__ loss) {
     if (threadIdx.x < s) part[threadIdx.x] += part[threadIdx.x + s];
     __syncthreads();
   }
-  if (threadIdx.x == 0) *loss = static_cast<float>(part[0] / static_cast<double>(T));
+  if (threadIdx.x == 0) *loss = static_cast<float>(scale * (part[0] / static_cast<double>(T)));
 }
 
 // Failure-detection probe: waits on a barrier that nothing arrives at.
@@ -378,8 +392,8 @@ WsLayout ws_layout(int64_t T, int64_t d, int64_t V, int K, int64_t chunk, int dt
 template <typename Elem>
 static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t d, int64_t V,
                           const float* t_vals, const int32_t* t_idx, int K, int64_t chunk,
-                          float tau, float* loss, float* lse, float* kl_rows, void* ws,
-                          cudaStream_t s, int num_sms, uint64_t limit_ns) {
+                          float tau, uint32_t flags, float* loss, float* lse, float* kl_rows,
+                          void* ws, cudaStream_t s, int num_sms, uint64_t limit_ns) {
   constexpr bool F32 = sizeof(Elem) == 4;
   constexpr int BK = ElemCfg<Elem>::BK;
   const WsLayout L = ws_layout(T, d, V, K, chunk, F32 ? KD_DTYPE_F32 : KD_DTYPE_BF16);
@@ -397,7 +411,8 @@ static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     const int64_t blocks64 = (T + PREP_WARPS - 1) / PREP_WARPS;
     const int blocks = static_cast<int>(blocks64 < 65535 * 16 ? blocks64 : 65535 * 16);
     prep_kernel<<<blocks, PREP_WARPS * 32, PREP_WARPS * PREP_MAXK * 8, s>>>(
-        t_vals, t_idx, T, K, V, inv_tau, idx_s, p_s, stats, status);
+        t_vals, t_idx, T, K, V, inv_tau, (flags & KD_KL_LOGPROB_CACHE) ? 1 : 0, idx_s, p_s, stats,
+        status);
     count_launch();
     if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
   }
@@ -438,7 +453,7 @@ static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     count_launch();
     if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
   }
-  mean_kernel<<<1, 1024, 0, s>>>(kl, T, loss);
+  mean_kernel<<<1, 1024, 0, s>>>(kl, T, loss_weight(tau, flags), loss);
   count_launch();
   if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
   return KD_OK;
@@ -447,9 +462,9 @@ static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
 template <typename Elem>
 static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, int64_t V,
                           const float* t_vals, const int32_t* t_idx, int K, int64_t chunk,
-                          float tau, const float* lse, const float* grad_loss, void* dH,
-                          float* dW, int accumulate, void* ws, cudaStream_t s, int num_sms,
-                          uint64_t limit_ns) {
+                          float tau, uint32_t flags, const float* lse, const float* grad_loss,
+                          void* dH, float* dW, int accumulate, void* ws, cudaStream_t s,
+                          int num_sms, uint64_t limit_ns) {
   constexpr bool F32 = sizeof(Elem) == 4;
   constexpr int BK = ElemCfg<Elem>::BK;
   constexpr int INNER = ROW_BYTES / sizeof(Elem);
@@ -467,7 +482,8 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     const int64_t blocks64 = (T + PREP_WARPS - 1) / PREP_WARPS;
     const int blocks = static_cast<int>(blocks64 < 65535 * 16 ? blocks64 : 65535 * 16);
     prep_kernel<<<blocks, PREP_WARPS * 32, PREP_WARPS * PREP_MAXK * 8, s>>>(
-        t_vals, t_idx, T, K, V, inv_tau, idx_s, p_s, stats, status);
+        t_vals, t_idx, T, K, V, inv_tau, (flags & KD_KL_LOGPROB_CACHE) ? 1 : 0, idx_s, p_s, stats,
+        status);
     count_launch();
     if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
   }
@@ -479,7 +495,8 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
   float* hpart = reinterpret_cast<float*>(w + L.hpart);
   if (!make_out_map(&tHP_out, hpart, true, d, KD_DH_MAX_SPLIT * L.rows_pad, d)) return KD_ERR_CUDA;
   const float zscale = 1.4426950408889634f * inv_tau;
-  const float inv_T_tau = static_cast<float>(1.0 / (static_cast<double>(T) * tau));
+  const float inv_T_tau =
+      static_cast<float>(loss_weight(tau, flags) / (static_cast<double>(T) * tau));
   // dz of KD_DW_GROUP consecutive chunks is kept side by side, so that dW is
   // updated once per group with K = the group's rows (halving dW's
   // read-modify-write traffic); dz and dH are formed chunk by chunk.
@@ -587,24 +604,25 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
 
 kd_status fused_fwd(const void* h, const void* W, int dtype, int64_t T, int64_t d, int64_t V,
                     const float* t_vals, const int32_t* t_idx, int K, int64_t chunk, float tau,
-                    float* loss, float* lse, float* kl_rows, void* ws, cudaStream_t s,
-                    int num_sms, uint64_t limit_ns) {
+                    uint32_t flags, float* loss, float* lse, float* kl_rows, void* ws,
+                    cudaStream_t s, int num_sms, uint64_t limit_ns) {
   if (dtype == KD_DTYPE_F32)
-    return fwd_impl<float>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, loss, lse, kl_rows, ws,
-                           s, num_sms, limit_ns);
-  return fwd_impl<__nv_bfloat16>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, loss, lse,
+    return fwd_impl<float>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, flags, loss, lse,
+                           kl_rows, ws, s, num_sms, limit_ns);
+  return fwd_impl<__nv_bfloat16>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, flags, loss, lse,
                                  kl_rows, ws, s, num_sms, limit_ns);
 }
 
 kd_status fused_bwd(const void* h, const void* W, int dtype, int64_t T, int64_t d, int64_t V,
                     const float* t_vals, const int32_t* t_idx, int K, int64_t chunk, float tau,
-                    const float* lse, const float* grad_loss, void* dH, float* dW,
-                    int accumulate, void* ws, cudaStream_t s, int num_sms, uint64_t limit_ns) {
+                    uint32_t flags, const float* lse, const float* grad_loss, void* dH,
+                    float* dW, int accumulate, void* ws, cudaStream_t s, int num_sms,
+                    uint64_t limit_ns) {
   if (dtype == KD_DTYPE_F32)
-    return bwd_impl<float>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, lse, grad_loss, dH, dW,
-                           accumulate, ws, s, num_sms, limit_ns);
-  return bwd_impl<__nv_bfloat16>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, lse, grad_loss,
-                                 dH, dW, accumulate, ws, s, num_sms, limit_ns);
+    return bwd_impl<float>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, flags, lse, grad_loss,
+                           dH, dW, accumulate, ws, s, num_sms, limit_ns);
+  return bwd_impl<__nv_bfloat16>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, flags, lse,
+                                 grad_loss, dH, dW, accumulate, ws, s, num_sms, limit_ns);
 }
 
 cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t s) {

@@ -11,10 +11,13 @@ Single H200 GPU Can Now Do That Once Required Four Nodes": d=4096, V=131072):
 * output head ``W ~ N(0, 1/d)`` (nn.Linear layout ``[V, d]``, no bias);
 * teacher cache indices: K distinct uniform draws per row (Floyd's sampling);
 * teacher cache values ``~ N(0, 2)`` (variance 2) as float32 logits;
-* teacher logits for the cache build ``~ N(0, 3)`` (variance 3), rounded to bf16.
+* teacher logits for the cache build ``~ N(0, 3)`` (variance 3), rounded to bf16;
+* for a cache of full-vocabulary teacher log-probabilities: the same N(0, 2)
+  draws shifted per row so that the K cached probabilities sum to a row mass
+  ``S ~ U(0.3, 0.95)`` (the rest is the tail the cache dropped).
 
 Every tensor has its own stream: generator seed = ``seed * 1000 + tensor_id``
-with ids h=0, W=1, vals=2, idx=3, teacher logits=4.
+with ids h=0, W=1, vals=2, idx=3, teacher logits=4, row mass=5.
 """
 
 from __future__ import annotations
@@ -23,7 +26,7 @@ import math
 
 import torch
 
-TENSOR_IDS = {"h": 0, "W": 1, "vals": 2, "idx": 3, "logits": 4}
+TENSOR_IDS = {"h": 0, "W": 1, "vals": 2, "idx": 3, "logits": 4, "mass": 5}
 
 
 def _gen(seed: int, name: str, device) -> torch.Generator:
@@ -72,6 +75,16 @@ def make_loss_inputs(T: int, d: int, V: int, K: int, dtype=torch.bfloat16, seed:
     vals = _randn((T, K), math.sqrt(2.0), torch.float32, seed, "vals", device)
     idx = distinct_uniform_indices(T, V, K, seed, device)
     return h, W, vals, idx
+
+
+def make_logprob_cache(T: int, K: int, seed: int = 0, device="cpu", mass=(0.3, 0.95)):
+    """Teacher log-probabilities [T, K] f32 of K tokens that carry a row mass
+    S_t ~ U(mass) of a full-vocabulary distribution: log S_t plus the
+    log-softmax of N(0, 2) draws.  Returns (vals, S)."""
+    x = _randn((T, K), math.sqrt(2.0), torch.float32, seed, "vals", device)
+    g = _gen(seed, "mass", device)
+    S = torch.empty((T,), dtype=torch.float32, device=device).uniform_(mass[0], mass[1], generator=g)
+    return torch.log_softmax(x, dim=1) + torch.log(S)[:, None], S
 
 
 def make_teacher_logits(T: int, V: int, seed: int = 0, device="cpu", dtype=torch.bfloat16,

@@ -26,8 +26,11 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG_DIR), "include", "kd.h")
 KD_OK, KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_WORKSPACE = 0, 1, 2, 3
 KD_ERR_BAD_INDEX, KD_ERR_TIMEOUT, KD_ERR_CUDA = 4, 5, 6
 KD_DTYPE_F32, KD_DTYPE_BF16 = 0, 1
+KD_KL_LOGPROB_CACHE, KD_KL_TAU_SQUARED = 0x1, 0x2
+CACHE_KINDS = ("logits", "logprobs")
 
 _c_i64, _c_int, _c_sz, _c_vp, _c_u64 = ctypes.c_int64, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_uint64
+_c_u32 = ctypes.c_uint32
 
 _SIGNATURES = {
     "kd_status_string": (ctypes.c_char_p, [_c_int]),
@@ -40,6 +43,12 @@ _SIGNATURES = {
     "kd_fused_kl_bwd": (_c_int, [_c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp, _c_int,
                                  _c_i64, ctypes.c_float, _c_vp, _c_vp, _c_vp, _c_vp, _c_int, _c_vp,
                                  _c_sz, _c_vp]),
+    "kd_fused_kl_fwd_ex": (_c_int, [_c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp, _c_int,
+                                    _c_i64, ctypes.c_float, _c_u32, _c_vp, _c_vp, _c_vp, _c_vp, _c_sz,
+                                    _c_vp]),
+    "kd_fused_kl_bwd_ex": (_c_int, [_c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp, _c_int,
+                                    _c_i64, ctypes.c_float, _c_u32, _c_vp, _c_vp, _c_vp, _c_vp, _c_int,
+                                    _c_vp, _c_sz, _c_vp]),
     "kd_read_device_status": (_c_int, [_c_vp, _c_vp]),
     "kd_set_wait_limit_ns": (_c_int, [_c_u64]),
     "kd_debug_wait_probe": (_c_int, [_c_vp, _c_sz, _c_u64, _c_vp]),
@@ -118,6 +127,19 @@ def kd_fused_kl_bwd(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, 
                     dW, accumulate_dW, ws, ws_bytes, stream):
     return load().kd_fused_kl_bwd(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, lse,
                                   grad_loss, dH, dW, accumulate_dW, ws, ws_bytes, stream)
+
+
+def kd_fused_kl_fwd_ex(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, flags, loss, lse,
+                       kl_rows, ws, ws_bytes, stream):
+    return load().kd_fused_kl_fwd_ex(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature,
+                                     flags, loss, lse, kl_rows, ws, ws_bytes, stream)
+
+
+def kd_fused_kl_bwd_ex(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, flags, lse,
+                       grad_loss, dH, dW, accumulate_dW, ws, ws_bytes, stream):
+    return load().kd_fused_kl_bwd_ex(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature,
+                                     flags, lse, grad_loss, dH, dW, accumulate_dW, ws, ws_bytes,
+                                     stream)
 
 
 def kd_fused_kl_fwd_noalloc(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, loss, lse,
@@ -239,58 +261,76 @@ def workspace_for(h: torch.Tensor, W: torch.Tensor, K: int, chunk: int) -> torch
     return alloc_workspace(kd_fused_kl_workspace_size(T, d, V, K, chunk, _dtype_code(h)), h.device)
 
 
+def kl_flags(cache: str = "logits", tau_squared: bool = False) -> int:
+    """The C ABI's flag bits for a cache kind ("logits": renormalised top-K
+    logits; "logprobs": full-vocabulary teacher log-probabilities, S <= 1) and
+    the optional tau^2 factor."""
+    if cache not in CACHE_KINDS:
+        raise ValueError(f"cache must be one of {CACHE_KINDS}")
+    return (KD_KL_LOGPROB_CACHE if cache == "logprobs" else 0) | (KD_KL_TAU_SQUARED if tau_squared else 0)
+
+
 def fused_kl_fwd(h, W, t_vals, t_idx, chunk: int, temperature: float = 1.0, ws=None,
-                 kl_rows: bool = False, stream=None):
+                 kl_rows: bool = False, stream=None, cache: str = "logits",
+                 tau_squared: bool = False):
     """Returns (loss [] f32, lse [T] f32, kl [T] f32 or None, ws)."""
     for t in (h, W, t_vals, t_idx):
         assert t.is_cuda and t.is_contiguous()
     T, d = h.shape
     V = W.shape[0]
     K = t_vals.shape[1]
+    flags = kl_flags(cache, tau_squared)
     if ws is None:
         ws = workspace_for(h, W, K, chunk)
     loss = torch.empty((), dtype=torch.float32, device=h.device)
     lse = torch.empty((T,), dtype=torch.float32, device=h.device)
     kl = torch.empty((T,), dtype=torch.float32, device=h.device) if kl_rows else None
-    _check(kd_fused_kl_fwd(h.data_ptr(), W.data_ptr(), _dtype_code(h), T, d, V, t_vals.data_ptr(),
-                           t_idx.data_ptr(), K, chunk, float(temperature), loss.data_ptr(),
-                           lse.data_ptr(), _ptr(kl), ws.data_ptr(), ws.numel(), _stream(stream)),
-           "kd_fused_kl_fwd")
+    _check(kd_fused_kl_fwd_ex(h.data_ptr(), W.data_ptr(), _dtype_code(h), T, d, V,
+                              t_vals.data_ptr(), t_idx.data_ptr(), K, chunk, float(temperature),
+                              flags, loss.data_ptr(), lse.data_ptr(), _ptr(kl), ws.data_ptr(),
+                              ws.numel(), _stream(stream)),
+           "kd_fused_kl_fwd_ex")
     return loss, lse, kl, ws
 
 
 def fused_kl_bwd(h, W, t_vals, t_idx, lse, chunk: int, temperature: float = 1.0, grad_loss=None,
-                 ws=None, dH=None, dW=None, accumulate_dW: bool = False, stream=None):
+                 ws=None, dH=None, dW=None, accumulate_dW: bool = False, stream=None,
+                 cache: str = "logits", tau_squared: bool = False):
     """Returns (dH [T,d] dtype of h, dW [V,d] f32, ws)."""
     T, d = h.shape
     V = W.shape[0]
     K = t_vals.shape[1]
+    flags = kl_flags(cache, tau_squared)
     if ws is None:
         ws = workspace_for(h, W, K, chunk)
     if dH is None:
         dH = torch.empty_like(h)
     if dW is None:
         dW = torch.empty((V, d), dtype=torch.float32, device=h.device)
-    _check(kd_fused_kl_bwd(h.data_ptr(), W.data_ptr(), _dtype_code(h), T, d, V, t_vals.data_ptr(),
-                           t_idx.data_ptr(), K, chunk, float(temperature), lse.data_ptr(),
-                           _ptr(grad_loss), dH.data_ptr(), dW.data_ptr(), int(accumulate_dW),
-                           ws.data_ptr(), ws.numel(), _stream(stream)),
-           "kd_fused_kl_bwd")
+    _check(kd_fused_kl_bwd_ex(h.data_ptr(), W.data_ptr(), _dtype_code(h), T, d, V,
+                              t_vals.data_ptr(), t_idx.data_ptr(), K, chunk, float(temperature),
+                              flags, lse.data_ptr(), _ptr(grad_loss), dH.data_ptr(), dW.data_ptr(),
+                              int(accumulate_dW), ws.data_ptr(), ws.numel(), _stream(stream)),
+           "kd_fused_kl_bwd_ex")
     return dH, dW, ws
 
 
 class FusedTopKKLLoss(torch.autograd.Function):
-    """Drop-in loss: forward = kd_fused_kl_fwd, backward = kd_fused_kl_bwd.
+    """Drop-in loss: forward = kd_fused_kl_fwd_ex, backward = kd_fused_kl_bwd_ex.
 
-    ``loss = FusedTopKKLLoss.apply(h, W, t_vals, t_idx, chunk, temperature)``;
-    gradients flow to h and W (W's gradient is returned in W's dtype).
+    ``loss = FusedTopKKLLoss.apply(h, W, t_vals, t_idx, chunk, temperature)``,
+    optionally followed by ``cache`` ("logits" or "logprobs") and
+    ``tau_squared``; gradients flow to h and W (W's gradient is returned in
+    W's dtype).
     """
 
     @staticmethod
-    def forward(ctx, h, W, t_vals, t_idx, chunk, temperature):
-        loss, lse, _, ws = fused_kl_fwd(h, W, t_vals, t_idx, chunk, temperature)
+    def forward(ctx, h, W, t_vals, t_idx, chunk, temperature, cache="logits", tau_squared=False):
+        loss, lse, _, ws = fused_kl_fwd(h, W, t_vals, t_idx, chunk, temperature, cache=cache,
+                                        tau_squared=tau_squared)
         ctx.save_for_backward(h, W, t_vals, t_idx, lse)
         ctx.chunk, ctx.temperature, ctx.ws = chunk, temperature, ws
+        ctx.cache, ctx.tau_squared = cache, tau_squared
         return loss
 
     @staticmethod
@@ -298,5 +338,6 @@ class FusedTopKKLLoss(torch.autograd.Function):
         h, W, t_vals, t_idx, lse = ctx.saved_tensors
         g = g.to(torch.float32).contiguous()
         dH, dW, _ = fused_kl_bwd(h, W, t_vals, t_idx, lse, ctx.chunk, ctx.temperature,
-                                 grad_loss=g, ws=ctx.ws)
-        return dH, dW.to(W.dtype), None, None, None, None
+                                 grad_loss=g, ws=ctx.ws, cache=ctx.cache,
+                                 tau_squared=ctx.tau_squared)
+        return dH, dW.to(W.dtype), None, None, None, None, None, None

@@ -141,6 +141,44 @@ kd_status kd_fused_kl_bwd(const void* h, const void* W, int dtype,
                           void* dH, float* dW, int accumulate_dW,
                           void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------ */
+/* Variants of the same objective, selected by `flags` (bitwise OR):        */
+/* ------------------------------------------------------------------------ */
+
+/* t_vals hold the teacher's log-probabilities from a softmax over the FULL
+ * vocabulary (at whatever temperature the teacher was run), not logits.
+ * p_tk = exp(t_vals[t,k]) is used as given, with no renormalisation and no
+ * temperature, so S_t = sum_k p_tk may be below 1 (the mass of the tokens the
+ * cache dropped).  The loss and gradient formulas above hold with this p:
+ * KL_t = sum_k p_tk (t_vals[t,k] - a_{t, t_idx[t,k]} + LSE_t), and dz keeps
+ * its S_t softmax - p form.  [DD] "The two changes" caches the teacher's top-K
+ * entries; this flag reads such a cache as probabilities of the full teacher
+ * distribution. */
+#define KD_KL_LOGPROB_CACHE 0x1u
+/* Multiply the loss and every gradient by tau^2 (the usual temperature
+ * compensation of distillation).  kl_rows stays the unscaled KL_t. */
+#define KD_KL_TAU_SQUARED 0x2u
+#define KD_KL_KNOWN_FLAGS (KD_KL_LOGPROB_CACHE | KD_KL_TAU_SQUARED)
+
+/* kd_fused_kl_fwd / kd_fused_kl_bwd with `flags`; flags == 0 is exactly the
+ * plain calls.  Pass the same flags to the forward and to the backward of one
+ * step (the backward re-derives p from t_vals).  Unknown bits return
+ * KD_ERR_INVALID_ARG and launch nothing. */
+kd_status kd_fused_kl_fwd_ex(const void* h, const void* W, int dtype,
+                             int64_t T, int64_t d, int64_t V,
+                             const float* t_vals, const int32_t* t_idx, int K,
+                             int64_t chunk, float temperature, uint32_t flags,
+                             float* loss, float* lse, float* kl_rows,
+                             void* ws, size_t ws_bytes, void* stream);
+
+kd_status kd_fused_kl_bwd_ex(const void* h, const void* W, int dtype,
+                             int64_t T, int64_t d, int64_t V,
+                             const float* t_vals, const int32_t* t_idx, int K,
+                             int64_t chunk, float temperature, uint32_t flags,
+                             const float* lse, const float* grad_loss,
+                             void* dH, float* dW, int accumulate_dW,
+                             void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, then returns the device status recorded in `ws`
  * (KD_OK, KD_ERR_BAD_INDEX or KD_ERR_TIMEOUT), or KD_ERR_CUDA. */
 kd_status kd_read_device_status(const void* ws, void* stream);

@@ -133,6 +133,48 @@ def test_bwd_output_pointers(lib):
     assert _bwd(lse=None) == kd.KD_ERR_INVALID_ARG
 
 
+def _fwd_ex(flags, **kw):
+    a = dict(h=FAKE, W=FAKE, dtype=kd.KD_DTYPE_BF16, T=256, d=256, V=4096, vals=FAKE, idx=FAKE,
+             K=16, chunk=64, tau=1.0, loss=FAKE, lse=FAKE, kl=None, ws=FAKE, ws_bytes=1 << 40,
+             stream=None)
+    a.update(kw)
+    return kd.kd_fused_kl_fwd_ex(a["h"], a["W"], a["dtype"], a["T"], a["d"], a["V"], a["vals"],
+                                 a["idx"], a["K"], a["chunk"], a["tau"], flags, a["loss"], a["lse"],
+                                 a["kl"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def _bwd_ex(flags, **kw):
+    a = dict(h=FAKE, W=FAKE, dtype=kd.KD_DTYPE_BF16, T=256, d=256, V=4096, vals=FAKE, idx=FAKE,
+             K=16, chunk=64, tau=1.0, lse=FAKE, g=None, dH=FAKE, dW=FAKE, acc=0, ws=FAKE,
+             ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return kd.kd_fused_kl_bwd_ex(a["h"], a["W"], a["dtype"], a["T"], a["d"], a["V"], a["vals"],
+                                 a["idx"], a["K"], a["chunk"], a["tau"], flags, a["lse"], a["g"],
+                                 a["dH"], a["dW"], a["acc"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("call", [_fwd_ex, _bwd_ex])
+def test_variant_flags_validation(lib, call):
+    E = kd
+    for bad in (0x4, 0x80000000, 0xFFFFFFFF, kd.KD_KL_LOGPROB_CACHE | 0x10):
+        assert call(bad) == E.KD_ERR_INVALID_ARG
+    # the shared checks still come first for valid flags
+    for ok in (0, kd.KD_KL_LOGPROB_CACHE, kd.KD_KL_TAU_SQUARED, 3):
+        assert call(ok, h=None) == E.KD_ERR_INVALID_ARG
+        assert call(ok, tau=0.0) == E.KD_ERR_INVALID_ARG
+        assert call(ok, d=12) == E.KD_ERR_UNSUPPORTED
+        assert call(ok, ws_bytes=1024) == E.KD_ERR_WORKSPACE
+
+
+def test_kl_flags_helper():
+    assert kd.kl_flags() == 0
+    assert kd.kl_flags("logprobs") == kd.KD_KL_LOGPROB_CACHE
+    assert kd.kl_flags("logits", True) == kd.KD_KL_TAU_SQUARED
+    assert kd.kl_flags("logprobs", True) == 3
+    with pytest.raises(ValueError):
+        kd.kl_flags("probs")
+
+
 def test_debug_api_validation(lib):
     assert kd.kd_set_wait_limit_ns(10) == kd.KD_ERR_INVALID_ARG
     assert kd.kd_debug_wait_probe(None, 4096, 10 ** 6, None) == kd.KD_ERR_INVALID_ARG

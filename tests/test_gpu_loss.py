@@ -25,25 +25,31 @@ LOSS_RTOL = 1e-3
 GRAD_TOL = 2e-2
 
 
-def _run(T, d, V, K, chunk, dtype, tau=1.0, g=None, seed=0, acc_init=None):
+def _run(T, d, V, K, chunk, dtype, tau=1.0, g=None, seed=0, acc_init=None, cache="logits",
+         tau_sq=False):
     h, W, vals, idx = inputs.make_loss_inputs(T, d, V, K, dtype=dtype, seed=seed, device="cuda")
-    loss, lse, kl, ws = kd.fused_kl_fwd(h, W, vals, idx, chunk, tau, kl_rows=True)
+    if cache == "logprobs":
+        vals, _ = inputs.make_logprob_cache(T, K, seed=seed, device="cuda")
+    var = dict(cache=cache, tau_squared=tau_sq)
+    loss, lse, kl, ws = kd.fused_kl_fwd(h, W, vals, idx, chunk, tau, kl_rows=True, **var)
     gl = None if g is None else torch.tensor(g, dtype=torch.float32, device="cuda")
     dW0 = None
     if acc_init is not None:
         dW0 = torch.full((V, d), acc_init, dtype=torch.float32, device="cuda")
     dH, dW, _ = kd.fused_kl_bwd(h, W, vals, idx, lse, chunk, tau, grad_loss=gl, ws=ws, dW=dW0,
-                                accumulate_dW=acc_init is not None)
+                                accumulate_dW=acc_init is not None, **var)
     torch.cuda.synchronize()
     assert kd.read_device_status(ws) == kd.KD_OK
-    return dict(h=h, W=W, vals=vals, idx=idx, loss=loss, lse=lse, kl=kl, dH=dH, dW=dW)
+    return dict(h=h, W=W, vals=vals, idx=idx, loss=loss, lse=lse, kl=kl, dH=dH, dW=dW,
+                cache=cache, tau_sq=tau_sq)
 
 
 def _full_parity(r, tau=1.0, g=1.0, lse_tol=1e-3, acc_init=None):
     h, W = to_np_exact(r["h"]), to_np_exact(r["W"])
     vals, idx = r["vals"].cpu().numpy(), r["idx"].cpu().numpy()
-    loss, lse, kl = oracle.forward(h, W, vals, idx, tau)
-    dH, dW = oracle.backward(h, W, vals, idx, tau, g)
+    var = dict(cache=r["cache"], tau_sq=r["tau_sq"])
+    loss, lse, kl = oracle.forward(h, W, vals, idx, tau, **var)
+    dH, dW = oracle.backward(h, W, vals, idx, tau, g, **var)
     if acc_init is not None:
         dW = dW + acc_init
     gl = float(r["loss"].item())
@@ -79,6 +85,52 @@ def test_temperature_grad_scale_and_accumulate():
     require_gpu()
     r = _run(200, 128, 3000, 20, 64, torch.bfloat16, tau=2.0, g=3.0, acc_init=0.25)
     _full_parity(r, tau=2.0, g=3.0, acc_init=0.25)
+
+
+@pytest.mark.parametrize("T,d,V,K,chunk,dtype,tau,g,tau_sq", [
+    (300, 200, 5000, 16, 100, torch.bfloat16, 1.0, None, False),
+    (256, 256, 4096, 16, 64, torch.float32, 1.5, 2.0, False),
+    (520, 264, 2304, 100, 512, torch.bfloat16, 2.0, 0.5, True),
+])
+def test_logprob_cache_parity(T, d, V, K, chunk, dtype, tau, g, tau_sq):
+    """Cache of full-vocabulary teacher log-probabilities (S < 1, no
+    renormalisation; tau scales the student only)."""
+    require_gpu()
+    r = _run(T, d, V, K, chunk, dtype, tau=tau, g=g, seed=T + 1, cache="logprobs", tau_sq=tau_sq)
+    S = torch.exp(r["vals"]).sum(dim=1)
+    assert float(S.max()) < 0.96 and float(S.min()) > 0.29
+    _full_parity(r, tau=tau, g=1.0 if g is None else g,
+                 lse_tol=5e-3 if dtype == torch.float32 else 1e-3)
+
+
+def test_tau_squared_parity():
+    require_gpu()
+    r = _run(200, 128, 3000, 20, 64, torch.bfloat16, tau=2.0, g=0.5, tau_sq=True, acc_init=-0.5)
+    _full_parity(r, tau=2.0, g=0.5, acc_init=-0.5)
+
+
+def test_flags_zero_is_the_plain_entry_point_bitwise():
+    """kd_fused_kl_fwd_ex / _bwd_ex with flags = 0 are the plain calls."""
+    require_gpu()
+    T, d, V, K, chunk = 200, 128, 3000, 20, 64
+    h, W, vals, idx = inputs.make_loss_inputs(T, d, V, K, dtype=torch.bfloat16, seed=8,
+                                              device="cuda")
+    loss_ex, lse_ex, _, ws = kd.fused_kl_fwd(h, W, vals, idx, chunk, 1.3)
+    dH_ex, dW_ex, _ = kd.fused_kl_bwd(h, W, vals, idx, lse_ex, chunk, 1.3, ws=ws)
+    loss = torch.empty((), dtype=torch.float32, device="cuda")
+    lse = torch.empty((T,), dtype=torch.float32, device="cuda")
+    dH, dW = torch.empty_like(h), torch.empty((V, d), dtype=torch.float32, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    assert kd.kd_fused_kl_fwd(h.data_ptr(), W.data_ptr(), kd.KD_DTYPE_BF16, T, d, V,
+                              vals.data_ptr(), idx.data_ptr(), K, chunk, 1.3, loss.data_ptr(),
+                              lse.data_ptr(), None, ws.data_ptr(), ws.numel(), s) == kd.KD_OK
+    assert kd.kd_fused_kl_bwd(h.data_ptr(), W.data_ptr(), kd.KD_DTYPE_BF16, T, d, V,
+                              vals.data_ptr(), idx.data_ptr(), K, chunk, 1.3, lse.data_ptr(), None,
+                              dH.data_ptr(), dW.data_ptr(), 0, ws.data_ptr(), ws.numel(),
+                              s) == kd.KD_OK
+    torch.cuda.synchronize()
+    assert torch.equal(loss, loss_ex) and torch.equal(lse, lse_ex)
+    assert torch.equal(dH, dH_ex) and torch.equal(dW, dW_ex)
 
 
 def test_chunk_invariance_bitwise():
@@ -153,6 +205,49 @@ def test_autograd_function():
     dH, dW = oracle.backward(hn, Wn, vals.cpu().numpy(), idx.cpu().numpy(), 1.0, 2.0)
     assert rel_maxabs(h.grad.float().cpu().numpy(), dH) <= GRAD_TOL
     assert rel_maxabs(W.grad.float().cpu().numpy(), dW) <= GRAD_TOL
+
+
+def test_autograd_function_logprob_cache_tau_squared():
+    require_gpu()
+    T, d, V, K = 96, 64, 777, 10
+    h, W, _, idx = inputs.make_loss_inputs(T, d, V, K, dtype=torch.bfloat16, seed=4, device="cuda")
+    vals, _ = inputs.make_logprob_cache(T, K, seed=4, device="cuda")
+    h.requires_grad_(True)
+    W.requires_grad_(True)
+    loss = kd.FusedTopKKLLoss.apply(h, W, vals, idx, 40, 1.5, "logprobs", True)
+    (0.75 * loss).backward()
+    torch.cuda.synchronize()
+    hn, Wn = to_np_exact(h), to_np_exact(W)
+    v, i = vals.cpu().numpy(), idx.cpu().numpy()
+    lo, _, _ = oracle.forward(hn, Wn, v, i, 1.5, cache="logprobs", tau_sq=True)
+    assert abs(loss.item() - lo) <= LOSS_RTOL * abs(lo)
+    dH, dW = oracle.backward(hn, Wn, v, i, 1.5, 0.75, cache="logprobs", tau_sq=True)
+    assert rel_maxabs(h.grad.float().cpu().numpy(), dH) <= GRAD_TOL
+    assert rel_maxabs(W.grad.float().cpu().numpy(), dW) <= GRAD_TOL
+
+
+def test_chain_topk_build_then_loss():
+    """The offline pipeline end to end: teacher logits [T, V] -> kd_topk_build
+    -> cache -> fused forward and backward, against the oracle's own top-K and
+    loss on the same teacher logits."""
+    require_gpu()
+    T, d, V, K, chunk = 160, 96, 3000, 20, 64
+    h, W, _, _ = inputs.make_loss_inputs(T, d, V, K, dtype=torch.bfloat16, seed=6, device="cuda")
+    x = inputs.make_teacher_logits(T, V, seed=6, device="cuda")
+    vals, idx = kd.topk_build(x, K)
+    loss, lse, _, ws = kd.fused_kl_fwd(h, W, vals, idx, chunk, 1.0)
+    dH, dW, _ = kd.fused_kl_bwd(h, W, vals, idx, lse, chunk, 1.0, ws=ws)
+    torch.cuda.synchronize()
+    assert kd.read_device_status(ws) == kd.KD_OK
+    ov, oi = oracle.topk_rows(to_np_exact(x), K)
+    assert np.array_equal(idx.cpu().numpy(), oi)
+    assert np.array_equal(vals.cpu().numpy().view(np.uint32), ov.view(np.uint32))
+    hn, Wn = to_np_exact(h), to_np_exact(W)
+    lo, _, _ = oracle.forward(hn, Wn, ov, oi, 1.0)
+    assert abs(loss.item() - lo) <= LOSS_RTOL * abs(lo)
+    dHo, dWo = oracle.backward(hn, Wn, ov, oi, 1.0)
+    assert rel_maxabs(dH.float().cpu().numpy(), dHo) <= GRAD_TOL
+    assert rel_maxabs(dW.cpu().numpy(), dWo) <= GRAD_TOL
 
 
 # ------------------------------------------------------------------ full-size
