@@ -219,19 +219,28 @@ __device__ __forceinline__ void offer8(TopkSmem& sm, uint4 q, uint32_t base, flo
   }
 }
 
-// Largest of the 8 bf16 values in q (NaNs ignored), as a float.
-__device__ __forceinline__ float max8_bf16(uint4 q) {
-  const __nv_bfloat162 a = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&q.x),
-                                   *reinterpret_cast<__nv_bfloat162*>(&q.y));
-  const __nv_bfloat162 b = __hmax2(*reinterpret_cast<__nv_bfloat162*>(&q.z),
-                                   *reinterpret_cast<__nv_bfloat162*>(&q.w));
-  const __nv_bfloat162 c = __hmax2(a, b);
-  return fmaxf(__low2float(c), __high2float(c));
+__device__ __forceinline__ __nv_bfloat162 as_bf162(uint32_t x) {
+  return *reinterpret_cast<__nv_bfloat162*>(&x);
 }
 
-// The streaming pass: every element of the row meets the threshold once.  A
-// 16-byte vector is first screened by its maximum (three packed max ops and
-// one compare); only vectors that may hold a survivor take the exact path.
+// Packed maximum of the 8 bf16 values in q: NaN inputs are ignored by
+// max.bf16x2 (the other operand is returned), so a NaN survives only where
+// both operands are NaN.
+__device__ __forceinline__ __nv_bfloat162 max8_packed(uint4 q) {
+  return __hmax2(__hmax2(as_bf162(q.x), as_bf162(q.y)), __hmax2(as_bf162(q.z), as_bf162(q.w)));
+}
+
+// True if some element of the pair is >= tb (a NaN compares false).
+__device__ __forceinline__ bool any_ge(__nv_bfloat162 m, __nv_bfloat16 tb) {
+  return __hge(__hmax(__low2bfloat16(m), __high2bfloat16(m)), tb);
+}
+
+// The streaming pass: every element of the row meets the threshold once.
+// Each thread holds TK_UNROLL 16-byte vectors (64 elements) in flight; one
+// packed max tree over all of them and one bf16 compare screen the group, and
+// only a group that may hold a survivor (usually one vector of it) takes the
+// exact per-vector path.  tf is a bf16 value (or -inf / 0), so comparing in
+// bf16 is exact.
 __device__ __forceinline__ void stream_survivors(TopkSmem& sm, const uint16_t* __restrict__ row,
                                                  int64_t V, float tf, bool take_all) {
   const uintptr_t addr = reinterpret_cast<uintptr_t>(row);
@@ -241,19 +250,25 @@ __device__ __forceinline__ void stream_survivors(TopkSmem& sm, const uint16_t* _
     offer(sm, row[i], static_cast<uint32_t>(i), tf, take_all);
   const int64_t nvec = (V - head) >> 3;
   const uint4* vp = reinterpret_cast<const uint4*>(row + head);
+  const __nv_bfloat16 tb = __float2bfloat16_rn(tf);
   for (int64_t j0 = threadIdx.x; j0 < nvec; j0 += TK_THREADS * TK_UNROLL) {
     uint4 q[TK_UNROLL];
 #pragma unroll
     for (int u = 0; u < TK_UNROLL; ++u) {
       const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
       q[u] = j < nvec ? __ldcs(vp + j) : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u,
-                                                   0xFF80FF80u);   // -inf: never passes
+                                                   0xFF80FF80u);   // -inf
     }
+    __nv_bfloat162 m = max8_packed(q[0]);
 #pragma unroll
-    for (int u = 0; u < TK_UNROLL; ++u) {
-      const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
-      if (j < nvec && (take_all || max8_bf16(q[u]) >= tf))
-        offer8(sm, q[u], static_cast<uint32_t>(head + (j << 3)), tf, take_all);
+    for (int u = 1; u < TK_UNROLL; ++u) m = __hmax2(m, max8_packed(q[u]));
+    if (take_all || any_ge(m, tb)) {
+#pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u) {
+        const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
+        if (j < nvec && (take_all || any_ge(max8_packed(q[u]), tb)))
+          offer8(sm, q[u], static_cast<uint32_t>(head + (j << 3)), tf, take_all);
+      }
     }
   }
   for (int64_t i = head + (nvec << 3) + threadIdx.x; i < V; i += TK_THREADS)
