@@ -51,7 +51,11 @@ __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
   return __uint_as_float((b & 0xFFFFu) << 16);
 }
 
+constexpr int TK_WARPS = TK_THREADS / 32;
+
 struct TopkSmem {
+  uint4 stage_q[TK_WARPS][32];        // per warp: screened vectors awaiting the exact test
+  uint32_t stage_base[TK_WARPS][32];  // and the row index of their first element
   uint32_t hist[TK_BINS];
   uint64_t cand[TK_CAND_CAP];
   uint64_t sel[TK_SEL_CAP];
@@ -236,11 +240,16 @@ __device__ __forceinline__ bool any_ge(__nv_bfloat162 m, __nv_bfloat16 tb) {
 }
 
 // The streaming pass: every element of the row meets the threshold once.
-// Each thread holds TK_UNROLL 16-byte vectors (64 elements) in flight; one
-// packed max tree over all of them and one bf16 compare screen the group, and
-// only a group that may hold a survivor (usually one vector of it) takes the
-// exact per-vector path.  tf is a bf16 value (or -inf / 0), so comparing in
-// bf16 is exact.
+// Each thread holds TK_UNROLL 16-byte vectors (64 elements) in flight, and each
+// vector is screened by its packed maximum (three max.bf16x2 and one bf16
+// compare; NaN operands are ignored by max.bf16x2, and tf is a bf16 value, or
+// -inf or 0, so the bf16 compare is exact).  A vector that may hold a survivor
+// is not tested on the spot, which would make the whole warp run the exact
+// test for one lane: its lane appends it to the warp's staging buffer
+// (position from a ballot), and once the buffer is full, and at the end, the
+// warp runs the exact test on up to 32 staged vectors at once, one per lane.
+// The row is walked in warp-uniform steps so that every lane takes part in
+// every ballot.
 __device__ __forceinline__ void stream_survivors(TopkSmem& sm, const uint16_t* __restrict__ row,
                                                  int64_t V, float tf, bool take_all) {
   const uintptr_t addr = reinterpret_cast<uintptr_t>(row);
@@ -251,7 +260,13 @@ __device__ __forceinline__ void stream_survivors(TopkSmem& sm, const uint16_t* _
   const int64_t nvec = (V - head) >> 3;
   const uint4* vp = reinterpret_cast<const uint4*>(row + head);
   const __nv_bfloat16 tb = __float2bfloat16_rn(tf);
-  for (int64_t j0 = threadIdx.x; j0 < nvec; j0 += TK_THREADS * TK_UNROLL) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const uint32_t lanes_below = (1u << lane) - 1u;
+  uint4* sq = sm.stage_q[wid];
+  uint32_t* sb = sm.stage_base[wid];
+  int cnt = 0;                                      // staged vectors (warp-uniform)
+  for (int64_t jb = 0; jb < nvec; jb += static_cast<int64_t>(TK_THREADS) * TK_UNROLL) {
+    const int64_t j0 = jb + threadIdx.x;
     uint4 q[TK_UNROLL];
 #pragma unroll
     for (int u = 0; u < TK_UNROLL; ++u) {
@@ -259,18 +274,31 @@ __device__ __forceinline__ void stream_survivors(TopkSmem& sm, const uint16_t* _
       q[u] = j < nvec ? __ldcs(vp + j) : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u,
                                                    0xFF80FF80u);   // -inf
     }
-    __nv_bfloat162 m = max8_packed(q[0]);
 #pragma unroll
-    for (int u = 1; u < TK_UNROLL; ++u) m = __hmax2(m, max8_packed(q[u]));
-    if (take_all || any_ge(m, tb)) {
-#pragma unroll
-      for (int u = 0; u < TK_UNROLL; ++u) {
-        const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
-        if (j < nvec && (take_all || any_ge(max8_packed(q[u]), tb)))
-          offer8(sm, q[u], static_cast<uint32_t>(head + (j << 3)), tf, take_all);
+    for (int u = 0; u < TK_UNROLL; ++u) {
+      const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
+      const bool pass = j < nvec && (take_all || any_ge(max8_packed(q[u]), tb));
+      const uint32_t b = __ballot_sync(0xffffffffu, pass);
+      if (b) {
+        const int nb = __popc(b);
+        if (cnt + nb > 32) {                        // buffer full: test what it holds
+          __syncwarp();
+          if (lane < cnt) offer8(sm, sq[lane], sb[lane], tf, take_all);
+          __syncwarp();
+          cnt = 0;
+        }
+        if (pass) {
+          const int pos = cnt + __popc(b & lanes_below);
+          sq[pos] = q[u];
+          sb[pos] = static_cast<uint32_t>(head + (j << 3));
+        }
+        cnt += nb;
       }
     }
   }
+  __syncwarp();
+  if (lane < cnt) offer8(sm, sq[lane], sb[lane], tf, take_all);
+  __syncwarp();
   for (int64_t i = head + (nvec << 3) + threadIdx.x; i < V; i += TK_THREADS)
     offer(sm, row[i], static_cast<uint32_t>(i), tf, take_all);
 }
