@@ -267,17 +267,31 @@ __device__ __forceinline__ void stream_survivors(TopkSmem& sm, const uint16_t* _
   int cnt = 0;                                      // staged vectors (warp-uniform)
   for (int64_t jb = 0; jb < nvec; jb += static_cast<int64_t>(TK_THREADS) * TK_UNROLL) {
     const int64_t j0 = jb + threadIdx.x;
+    const bool full = jb + static_cast<int64_t>(TK_THREADS) * TK_UNROLL <= nvec;  // warp-uniform
     uint4 q[TK_UNROLL];
+    if (full) {
+#pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u) q[u] = __ldcs(vp + j0 + u * TK_THREADS);
+    } else {
+#pragma unroll
+      for (int u = 0; u < TK_UNROLL; ++u) {
+        const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
+        q[u] = j < nvec ? __ldcs(vp + j) : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u,
+                                                     0xFF80FF80u);   // -inf
+      }
+    }
+    // The next step's vectors into L2 while this step's are screened (a hint:
+    // no registers held, nothing waits on it).
 #pragma unroll
     for (int u = 0; u < TK_UNROLL; ++u) {
-      const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
-      q[u] = j < nvec ? __ldcs(vp + j) : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u,
-                                                   0xFF80FF80u);   // -inf
+      const int64_t j = j0 + static_cast<int64_t>(TK_THREADS) * TK_UNROLL +
+                        static_cast<int64_t>(u) * TK_THREADS;
+      if (j < nvec) asm volatile("prefetch.global.L2 [%0];" ::"l"(vp + j));
     }
 #pragma unroll
     for (int u = 0; u < TK_UNROLL; ++u) {
       const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
-      const bool pass = j < nvec && (take_all || any_ge(max8_packed(q[u]), tb));
+      const bool pass = (full || j < nvec) && (take_all || any_ge(max8_packed(q[u]), tb));
       const uint32_t b = __ballot_sync(0xffffffffu, pass);
       if (b) {
         const int nb = __popc(b);
