@@ -133,8 +133,19 @@ def _cpu_setup(w, rows, seed=0):
     return W64, hn, xn
 
 
-def cpu_baseline(w, rows=0, steps=1):
-    """Oracle tokens/s on a bounded sample (rows positions per step)."""
+def _cpu_model():
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
+def cpu_baseline(w, rows=0, steps=1, single_core_rows=32):
+    """Oracle tokens/s on a bounded sample (rows positions per step), on all
+    host cores and, on a smaller sample, on one core."""
     if rows <= 0:
         rows = 16
     W64, hn, xn = _cpu_setup(w, rows)
@@ -142,10 +153,21 @@ def cpu_baseline(w, rows=0, steps=1):
     for _ in range(steps):
         _cpu_sample_step(W64, hn, xn, w["K"])
     dt = time.perf_counter() - t0
-    return {"value": rows * steps / dt, "unit": UNIT, "cores": _cpu_threads(), "kind": "oracle",
-            "sample": f"{rows} positions x {steps} step(s) of the {w['T']}-position batch: "
-                      f"fp64 top-K (full stable sort of V={w['V']}), forward and backward "
-                      f"(d={w['d']}); {dt:.2f} s"}
+    out = {"value": rows * steps / dt, "unit": UNIT, "cores": _cpu_threads(), "kind": "oracle",
+           "cpu_model": _cpu_model(), "nproc": os.cpu_count(),
+           "sample": f"{rows} positions x {steps} step(s) of the {w['T']}-position batch: "
+                     f"fp64 top-K (full stable sort of V={w['V']}), forward and backward "
+                     f"(d={w['d']}); {dt:.2f} s"}
+    if single_core_rows > 0:
+        from threadpoolctl import threadpool_limits
+        n1 = min(single_core_rows, rows)
+        with threadpool_limits(limits=1):
+            t0 = time.perf_counter()
+            _cpu_sample_step(W64, hn[:n1], xn[:n1], w["K"])
+            dt1 = time.perf_counter() - t0
+        out["single_core"] = {"value": n1 / dt1, "unit": UNIT, "cores": 1,
+                              "sample": f"{n1} positions of the same sample; {dt1:.2f} s"}
+    return out
 
 
 def run_reference(args, rank):
@@ -462,6 +484,8 @@ def sweep_memory(args):
     from chunked_kl_loss_chunk_b200 import inputs, kd
     kbuild.build()
     dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    torch.empty(1, device=dev)          # initialise the caching allocator
     d, V, K, chunk = 4096, 131072, 100, 4096
     out = []
     for T in (4096, 8192, 16384, 32768, 65536, 131072, 262144):
