@@ -81,6 +81,19 @@ def test_ragged_shapes(T, d, V, K, chunk, dtype):
     _full_parity(r, lse_tol=5e-3 if dtype == torch.float32 else 1e-3)
 
 
+@pytest.mark.parametrize("T,d,V,K,chunk,dtype", [
+    (1, 8, 40, 3, 1, torch.bfloat16),              # one position, minimum d
+    (33, 8, 300, 5, 1, torch.float32),             # chunk = 1: one launch per position
+    (5, 16, 1030, 1024, 2, torch.bfloat16),        # K at its maximum
+    (3, 4104, 513, 9, 7, torch.bfloat16),          # d > 4096 and not a multiple of 64, T < chunk
+    (40, 64, 1024, 1024, 40, torch.bfloat16),      # K = V = 1024
+])
+def test_edge_shapes(T, d, V, K, chunk, dtype):
+    require_gpu()
+    r = _run(T, d, V, K, chunk, dtype, seed=T + d)
+    _full_parity(r, lse_tol=5e-3 if dtype == torch.float32 else 1e-3)
+
+
 def test_temperature_grad_scale_and_accumulate():
     require_gpu()
     r = _run(200, 128, 3000, 20, 64, torch.bfloat16, tau=2.0, g=3.0, acc_init=0.25)
