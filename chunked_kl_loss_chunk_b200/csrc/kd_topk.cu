@@ -42,10 +42,22 @@ __device__ __forceinline__ uint32_t bf16_order_key(uint32_t b) {
   return (b & 0x8000u) ? (~b & 0xFFFFu) : (b | 0x8000u);
 }
 
-// Ascending order of this 64-bit composite = key descending, index ascending.
-__device__ __forceinline__ uint64_t composite(uint32_t key, uint32_t idx) {
-  return (static_cast<uint64_t>(0xFFFFu - key) << 32) | idx;
+// 64-bit candidate: (0xFFFF - key) in bits 48..63, the index (< 2^31) in bits
+// 16..46, the raw bf16 bits in bits 0..15.  Ascending order of composites is
+// key descending, then index ascending (indices are distinct within a row, so
+// the raw bits never decide); the raw bits give the exact output value without
+// reading the row again.
+__device__ __forceinline__ uint64_t composite(uint32_t key, uint32_t idx, uint32_t raw) {
+  return (static_cast<uint64_t>(0xFFFFu - key) << 48) | (static_cast<uint64_t>(idx) << 16) |
+         (raw & 0xFFFFu);
 }
+__device__ __forceinline__ uint32_t comp_key(uint64_t c) {
+  return 0xFFFFu - static_cast<uint32_t>(c >> 48);
+}
+__device__ __forceinline__ uint32_t comp_idx(uint64_t c) {
+  return static_cast<uint32_t>(c >> 16) & 0x7FFFFFFFu;
+}
+__device__ __forceinline__ uint32_t comp_raw(uint64_t c) { return static_cast<uint32_t>(c) & 0xFFFFu; }
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) {
   return __uint_as_float((b & 0xFFFFu) << 16);
@@ -66,6 +78,7 @@ struct TopkSmem {
   uint32_t thr_bin;
   uint32_t thr_above;
   uint32_t eq_base;
+  uint32_t wide;
 };
 
 // Exclusive block scan of one value per thread (TK_THREADS threads); also
@@ -198,7 +211,7 @@ __device__ __forceinline__ void offer(TopkSmem& sm, uint32_t bits, uint32_t i, f
                                      bool take_all) {
   if (take_all || bf16_bits_to_float(bits) >= tf) {
     const uint32_t pos = atomicAdd(&sm.n_cand, 1u);
-    if (pos < TK_CAND_CAP) sm.cand[pos] = composite(bf16_order_key(bits), i);
+    if (pos < TK_CAND_CAP) sm.cand[pos] = composite(bf16_order_key(bits), i, bits);
   }
 }
 
@@ -219,7 +232,7 @@ __device__ __forceinline__ void offer8(TopkSmem& sm, uint4 q, uint32_t base, flo
     m &= m - 1;
     const uint32_t bits = (w[b >> 1] >> ((b & 1) * 16)) & 0xFFFFu;
     const uint32_t pos = atomicAdd(&sm.n_cand, 1u);
-    if (pos < TK_CAND_CAP) sm.cand[pos] = composite(bf16_order_key(bits), base + b);
+    if (pos < TK_CAND_CAP) sm.cand[pos] = composite(bf16_order_key(bits), base + b, bits);
   }
 }
 
@@ -421,34 +434,62 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
 
     if (n >= static_cast<uint32_t>(K) && n <= static_cast<uint32_t>(TK_CAND_CAP)) {
       // ---- 3. exact select among survivors -------------------------------------
-      // (a) the exact K-th largest key among the survivors (4096-bin histogram
-      //     of key >> 4, then the 16 keys of the threshold bin);
-      for (int b = tid; b < TK_BINS; b += TK_THREADS) sm.hist[b] = 0u;
-      if (tid < 16) sm.hist16[tid] = 0u;
+      // (a) the exact K-th largest key among the survivors.  Every survivor's
+      //     key is >= L.  When they span fewer than TK_THREADS keys (the usual
+      //     case: few bf16 values lie near the top of a row) one histogram of
+      //     key - L, one bin per thread, and one block scan give it; otherwise
+      //     a 4096-bin histogram of key >> 4, then the 16 keys of the
+      //     threshold bin.
+      static_assert(TK_THREADS <= TK_BINS, "narrow histogram lives in hist");
+      if (tid == 0) {
+        sm.wide = 0u;
+        sm.n_sel = 0u;
+      }
+      sm.hist[tid] = 0u;
       __syncthreads();
-      for (int i = tid; i < static_cast<int>(n); i += TK_THREADS)
-        atomicAdd(&sm.hist[(0xFFFFu - static_cast<uint32_t>(sm.cand[i] >> 32)) >> 4], 1u);
-      __syncthreads();
-      find_threshold_bin(sm, static_cast<uint32_t>(K));
-      const uint32_t cb = sm.thr_bin;
       for (int i = tid; i < static_cast<int>(n); i += TK_THREADS) {
-        const uint32_t key = 0xFFFFu - static_cast<uint32_t>(sm.cand[i] >> 32);
-        if ((key >> 4) == cb) atomicAdd(&sm.hist16[key & 15u], 1u);
+        const uint32_t dk = comp_key(sm.cand[i]) - L;
+        if (dk < static_cast<uint32_t>(TK_THREADS))
+          atomicAdd(&sm.hist[TK_THREADS - 1 - dk], 1u);   // bin 0 = highest key
+        else
+          sm.wide = 1u;
       }
       __syncthreads();
-      if (tid == 0) {
-        uint32_t above = sm.thr_above, nib = 0, at = 0;
-        for (int j = 15; j >= 0; --j) {
-          if (above + sm.hist16[j] >= static_cast<uint32_t>(K)) {
-            nib = static_cast<uint32_t>(j);
-            at = sm.hist16[j];
-            break;
-          }
-          above += sm.hist16[j];
+      if (sm.wide == 0u) {
+        const uint32_t c = sm.hist[tid];
+        uint32_t total;
+        const uint32_t above = block_excl_scan(c, sm.warp_tot, total);  // keys above bin tid
+        if (above < static_cast<uint32_t>(K) && above + c >= static_cast<uint32_t>(K)) {
+          sm.thr_bin = L + static_cast<uint32_t>(TK_THREADS - 1 - tid);   // exact K-th key
+          sm.thr_above = above + c;                                      // survivors >= it
         }
-        sm.thr_bin = (cb << 4) | nib;     // exact K-th key
-        sm.thr_above = above + at;        // survivors with key >= it
-        sm.n_sel = 0;
+      } else {
+        for (int b = tid; b < TK_BINS; b += TK_THREADS) sm.hist[b] = 0u;
+        if (tid < 16) sm.hist16[tid] = 0u;
+        __syncthreads();
+        for (int i = tid; i < static_cast<int>(n); i += TK_THREADS)
+          atomicAdd(&sm.hist[comp_key(sm.cand[i]) >> 4], 1u);
+        __syncthreads();
+        find_threshold_bin(sm, static_cast<uint32_t>(K));
+        const uint32_t cb = sm.thr_bin;
+        for (int i = tid; i < static_cast<int>(n); i += TK_THREADS) {
+          const uint32_t key = comp_key(sm.cand[i]);
+          if ((key >> 4) == cb) atomicAdd(&sm.hist16[key & 15u], 1u);
+        }
+        __syncthreads();
+        if (tid == 0) {
+          uint32_t above = sm.thr_above, nib = 0, at = 0;
+          for (int j = 15; j >= 0; --j) {
+            if (above + sm.hist16[j] >= static_cast<uint32_t>(K)) {
+              nib = static_cast<uint32_t>(j);
+              at = sm.hist16[j];
+              break;
+            }
+            above += sm.hist16[j];
+          }
+          sm.thr_bin = (cb << 4) | nib;     // exact K-th key
+          sm.thr_above = above + at;        // survivors with key >= it
+        }
       }
       __syncthreads();
       const uint32_t Tk = sm.thr_bin;
@@ -457,7 +498,7 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
       if (compact) {
         for (int i = tid; i < static_cast<int>(n); i += TK_THREADS) {
           const uint64_t c = sm.cand[i];
-          if (0xFFFFu - static_cast<uint32_t>(c >> 32) >= Tk) sm.sel[atomicAdd(&sm.n_sel, 1u)] = c;
+          if (comp_key(c) >= Tk) sm.sel[atomicAdd(&sm.n_sel, 1u)] = c;
         }
         __syncthreads();
       }
@@ -469,11 +510,11 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
       for (int i = tid; i < ns; i += TK_THREADS) {
         const uint64_t c = set[i];
         int rank = 0;
+#pragma unroll 8
         for (int j = 0; j < ns; ++j) rank += set[j] < c ? 1 : 0;
         if (rank < K) {
-          const uint32_t idx = static_cast<uint32_t>(c);
-          out_idx[t * K + rank] = static_cast<int32_t>(idx);
-          out_vals[t * K + rank] = bf16_bits_to_float(row[idx]);
+          out_idx[t * K + rank] = static_cast<int32_t>(comp_idx(c));
+          out_vals[t * K + rank] = bf16_bits_to_float(comp_raw(c));
         }
       }
       __syncthreads();
@@ -503,7 +544,7 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
       const uint32_t b = key >> 4;
       if (b > b1) {
         const uint32_t pos = atomicAdd(&sm.n_sel, 1u);
-        sm.sel[pos] = composite(key, i);
+        sm.sel[pos] = composite(key, i, bits);
       } else if (b == b1) {
         atomicAdd(&sm.hist16[key & 15u], 1u);
       }
@@ -533,10 +574,11 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
       for (int u = 0; u < 8; ++u) {
         const int64_t i = i0 + u;
         if (i < V) {
-          const uint32_t key = bf16_order_key(row[i]);
+          const uint32_t bits = row[i];
+          const uint32_t key = bf16_order_key(bits);
           if ((key >> 4) == b1 && key > Tk) {
             const uint32_t pos = atomicAdd(&sm.n_sel, 1u);
-            sm.sel[pos] = composite(key, static_cast<uint32_t>(i));
+            sm.sel[pos] = composite(key, static_cast<uint32_t>(i), bits);
           } else if (key == Tk) {
             eq_mask |= 1u << u;
           }
@@ -551,7 +593,7 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
         if (eq_mask & (1u << u)) {
           if (r < need) {
             const uint32_t pos = atomicAdd(&sm.n_sel, 1u);
-            sm.sel[pos] = composite(Tk, static_cast<uint32_t>(i0 + u));
+            sm.sel[pos] = composite(Tk, static_cast<uint32_t>(i0 + u), row[i0 + u]);
           }
           ++r;
         }
@@ -566,9 +608,8 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
     bitonic_sort(sm.sel, np);
     for (int k = tid; k < K; k += TK_THREADS) {
       const uint64_t c = sm.sel[k];
-      const uint32_t i = static_cast<uint32_t>(c);
-      out_idx[t * K + k] = static_cast<int32_t>(i);
-      out_vals[t * K + k] = bf16_bits_to_float(row[i]);
+      out_idx[t * K + k] = static_cast<int32_t>(comp_idx(c));
+      out_vals[t * K + k] = bf16_bits_to_float(comp_raw(c));
     }
     __syncthreads();
   }
