@@ -113,6 +113,41 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_t
   return r;
 }
 
+// Warp 0 only: among 256 bin counts h[0..256), bin 0 holding the highest keys,
+// the bin b where the running count from bin 0 first reaches `target`
+// (1 <= target <= total).  Writes b, the count of bins before b and the count
+// of bins up to and including b.  h must be 16-byte aligned.
+__device__ __forceinline__ void find_bin_256(const uint32_t* h, uint32_t target, uint32_t* out_bin,
+                                             uint32_t* out_above, uint32_t* out_through) {
+  if (threadIdx.x >= 32) return;
+  const int lane = threadIdx.x;
+  const uint4 a = reinterpret_cast<const uint4*>(h)[2 * lane];
+  const uint4 b = reinterpret_cast<const uint4*>(h)[2 * lane + 1];
+  const uint32_t c[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  uint32_t sum = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) sum += c[j];
+  uint32_t incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  uint32_t run = incl - sum;
+  if (run < target && incl >= target) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (run + c[j] >= target) {
+        *out_bin = static_cast<uint32_t>(lane * 8 + j);
+        *out_above = run;
+        *out_through = run + c[j];
+        break;
+      }
+      run += c[j];
+    }
+  }
+}
+
 // Highest bin b with (count of bins > b) < target <= (count of bins >= b).
 // If the histogram holds fewer than `target` elements, returns bin 0.
 // Writes sm.thr_bin / sm.thr_above.
@@ -341,7 +376,11 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
     const uint16_t* row = logits + t * V;
 
     // ---- 1. sample threshold -------------------------------------------------
-    for (int b = tid; b < TK_BINS; b += TK_THREADS) sm.hist[b] = 0u;
+    // L = the key of the target-th largest sample element, found in two levels
+    // of 256 bins: the key's high byte, then its low byte inside the chosen
+    // high-byte bin (bin 0 holds the highest keys).
+    sm.hist[tid] = 0u;
+    sm.hist[TK_THREADS + tid] = 0u;
     if (tid == 0) {
       sm.n_cand = 0;
       sm.n_sel = 0;
@@ -380,8 +419,7 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
     }
 #pragma unroll
     for (int u = 0; u < SAMPLE_PER_THREAD; ++u)
-      if (skey[u] != 0xFFFFFFFFu) atomicAdd(&sm.hist[skey[u] >> 4], 1u);
-    if (tid < 16) sm.hist16[tid] = 0u;
+      if (skey[u] != 0xFFFFFFFFu) atomicAdd(&sm.hist[255u - (skey[u] >> 8)], 1u);
     __syncthreads();
     uint32_t target;
     if (S == V) {
@@ -392,26 +430,20 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
       target = static_cast<uint32_t>(ceil(want));
       if (target < 1u) target = 1u;
     }
-    find_threshold_bin(sm, target);
-    // Refine to the exact key of the target-th largest sample element: split
-    // the threshold bin into its 16 keys.
-    const uint32_t sb = sm.thr_bin, s_above = sm.thr_above;
+    // (target <= S: either S == V >= K, or V > 4096 >= 3K)
+    find_bin_256(sm.hist, target, &sm.thr_bin, &sm.thr_above, &sm.n_sel);
+    __syncthreads();
+    const uint32_t hb = 255u - sm.thr_bin;            // high byte of L
+    const uint32_t above_hb = sm.thr_above;
 #pragma unroll
     for (int u = 0; u < SAMPLE_PER_THREAD; ++u)
-      if (skey[u] != 0xFFFFFFFFu && (skey[u] >> 4) == sb) atomicAdd(&sm.hist16[skey[u] & 15u], 1u);
+      if (skey[u] != 0xFFFFFFFFu && (skey[u] >> 8) == hb)
+        atomicAdd(&sm.hist[TK_THREADS + 255u - (skey[u] & 255u)], 1u);
     __syncthreads();
-    uint32_t L = sb << 4;                 // candidate iff order key >= L
-    {
-      uint32_t above = s_above;
-      for (int j = 15; j >= 0; --j) {
-        above += sm.hist16[j];
-        if (above >= target) {
-          L = (sb << 4) | static_cast<uint32_t>(j);
-          break;
-        }
-      }
-    }
+    find_bin_256(sm.hist + TK_THREADS, target - above_hb, &sm.thr_bin, &sm.thr_above, &sm.n_sel);
     __syncthreads();
+    const uint32_t L = (hb << 8) | (255u - sm.thr_bin);   // candidate iff order key >= L
+    if (tid == 0) sm.n_sel = 0u;
     // Float threshold equivalent on non-NaN values: key >= L <=> x >= tf.
     float tf = 0.f;
     bool take_all = false;
@@ -456,12 +488,12 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
       }
       __syncthreads();
       if (sm.wide == 0u) {
-        const uint32_t c = sm.hist[tid];
-        uint32_t total;
-        const uint32_t above = block_excl_scan(c, sm.warp_tot, total);  // keys above bin tid
-        if (above < static_cast<uint32_t>(K) && above + c >= static_cast<uint32_t>(K)) {
-          sm.thr_bin = L + static_cast<uint32_t>(TK_THREADS - 1 - tid);   // exact K-th key
-          sm.thr_above = above + c;                                      // survivors >= it
+        uint32_t* res = sm.warp_tot;                 // scratch: bin, above, through
+        find_bin_256(sm.hist, static_cast<uint32_t>(K), &res[0], &res[1], &res[2]);
+        __syncthreads();
+        if (tid == 0) {
+          sm.thr_bin = L + static_cast<uint32_t>(TK_THREADS - 1) - res[0];   // exact K-th key
+          sm.thr_above = res[2];                                            // survivors >= it
         }
       } else {
         for (int b = tid; b < TK_BINS; b += TK_THREADS) sm.hist[b] = 0u;
