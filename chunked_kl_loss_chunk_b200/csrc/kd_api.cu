@@ -121,6 +121,9 @@ static kd_status validate_loss(const void* h, const void* W, int dtype, int64_t 
   if (d % 8 != 0 || K > KD_MAX_K || V >= (int64_t(1) << 31) - 256 ||
       d >= (int64_t(1) << 31) || T >= (int64_t(1) << 40))
     return KD_ERR_UNSUPPORTED;
+  // Rows per chunk: the backward contracts dW over two chunks' rows in one
+  // 32-bit GEMM extent.
+  if ((chunk < T ? chunk : T) > (int64_t(1) << 30)) return KD_ERR_UNSUPPORTED;
   if (ws_bytes < kd::ws_layout(T, d, V, K, chunk, dtype).total) return KD_ERR_WORKSPACE;
   return KD_OK;
 }

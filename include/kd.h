@@ -112,7 +112,8 @@ size_t kd_fused_kl_workspace_size(int64_t T, int64_t d, int64_t V, int K, int64_
  *   loss   float32 scalar    mean KL over the T positions
  *   lse    float32 [T]       LSE_t (keep it for kd_fused_kl_bwd)
  *   kl_rows float32 [T] or NULL   per-position KL_t
- * Requires d % 8 == 0, 1 <= K <= min(V, 1024), chunk >= 1, V < 2^31 - 256.
+ * Requires d % 8 == 0, 1 <= K <= min(V, 1024), chunk >= 1, V < 2^31 - 256,
+ * T < 2^40 and min(chunk, T) <= 2^30 (else KD_ERR_UNSUPPORTED).
  * Per-position results (lse, kl_rows) and the loss are bit-identical for every
  * `chunk`.
  */

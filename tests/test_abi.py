@@ -119,6 +119,9 @@ def test_loss_validation(lib, call):
     assert call(d=12) == E.KD_ERR_UNSUPPORTED               # d % 8 != 0
     assert call(K=1025) == E.KD_ERR_UNSUPPORTED             # K above the maximum
     assert call(ws_bytes=1024) == E.KD_ERR_WORKSPACE
+    assert call(T=1 << 40) == E.KD_ERR_UNSUPPORTED
+    assert call(T=(1 << 30) + 1, chunk=(1 << 30) + 1) == E.KD_ERR_UNSUPPORTED   # rows per chunk
+    assert call(T=(1 << 31), chunk=1 << 30, ws_bytes=1024) == E.KD_ERR_WORKSPACE   # 2^30 rows pass
 
 
 def test_fwd_output_pointers(lib):
