@@ -9,7 +9,7 @@
 
 namespace {
 
-uint64_t g_wait_limit_ns = 4000000000ull;  // 4 s
+std::atomic<uint64_t> g_wait_limit_ns{4000000000ull};  // 4 s; set from any host thread
 std::atomic<uint64_t> g_launches{0};
 
 struct Profile {
@@ -38,7 +38,7 @@ namespace kd {
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
-uint64_t wait_limit_ns() { return g_wait_limit_ns; }
+uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
 void profile_before(int kind, double flops, cudaStream_t s) {
   g_prof.armed = false;
@@ -143,7 +143,7 @@ kd_status kd_fused_kl_fwd_ex(const void* h, const void* W, int dtype, int64_t T,
   const int sms = num_sms_current();
   if (sms <= 0) return KD_ERR_CUDA;
   return kd::fused_fwd(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, flags, loss,
-                       lse, kl_rows, ws, static_cast<cudaStream_t>(stream), sms, g_wait_limit_ns);
+                       lse, kl_rows, ws, static_cast<cudaStream_t>(stream), sms, kd::wait_limit_ns());
 }
 
 kd_status kd_fused_kl_fwd(const void* h, const void* W, int dtype, int64_t T, int64_t d,
@@ -171,7 +171,7 @@ kd_status kd_fused_kl_bwd_ex(const void* h, const void* W, int dtype, int64_t T,
   if (sms <= 0) return KD_ERR_CUDA;
   return kd::fused_bwd(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, flags, lse,
                        grad_loss, dH, dW, accumulate_dW, ws, static_cast<cudaStream_t>(stream),
-                       sms, g_wait_limit_ns);
+                       sms, kd::wait_limit_ns());
 }
 
 kd_status kd_fused_kl_bwd(const void* h, const void* W, int dtype, int64_t T, int64_t d,
@@ -216,7 +216,7 @@ int kd_profile_detach(void) {
 
 kd_status kd_set_wait_limit_ns(uint64_t limit_ns) {
   if (limit_ns < 1000) return KD_ERR_INVALID_ARG;
-  g_wait_limit_ns = limit_ns;
+  g_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
   return KD_OK;
 }
 

@@ -11,6 +11,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "kd_gemm.cuh"
 #include "kd_gemm2.cuh"
 #include "kd_internal.h"
@@ -279,13 +281,19 @@ bool make_out_map(CUtensorMap* map, const void* base, bool f32, uint64_t inner, 
                   f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-// Clusters of two CTAs that can be resident at once for this kernel.
+// Clusters of two CTAs that can be resident at once for this kernel, cached
+// per device (atomics: calls may come from several host threads).
+constexpr int KD_MAX_DEVICES = 64;
 template <typename Kern>
 int max_pair_clusters(Kern kern, int num_sms) {
-  static int cached_dev = -1, cached = 0;
+  static std::atomic<int> cache[KD_MAX_DEVICES];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev == cached_dev && cached > 0) return cached;
+  const bool cacheable = dev >= 0 && dev < KD_MAX_DEVICES;
+  if (cacheable) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * (num_sms / 2));
   cfg.blockDim = dim3(GEMM_THREADS);
@@ -302,8 +310,7 @@ int max_pair_clusters(Kern kern, int num_sms) {
     cudaGetLastError();
     n = num_sms / 2;
   }
-  cached_dev = dev;
-  cached = n;
+  if (cacheable) cache[dev].store(n, std::memory_order_relaxed);
   return n;
 }
 
