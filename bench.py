@@ -143,12 +143,61 @@ def _cpu_model():
     return None
 
 
-def cpu_baseline(w, rows=0, steps=1, single_core_rows=32):
+def _cpu_from_gpu(gpu, rows):
+    """Host copies of `rows` evenly spaced positions of the bench's own batch
+    (exact bf16 bit patterns) and of the full output head, widened to fp64."""
+    import numpy as np
+    import torch
+    import oracle
+    T = gpu["h"].shape[0]
+    sel = np.unique(np.linspace(0, T - 1, min(rows, T)).round().astype(np.int64))
+    st = torch.as_tensor(sel, device=gpu["h"].device)
+
+    def bits(t):
+        t = t.detach().cpu().contiguous()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+    W64 = oracle.bf16_bits_to_f64(bits(gpu["W"])) if gpu["W"].dtype == torch.bfloat16 \
+        else gpu["W"].double().cpu().numpy()
+    return W64, bits(gpu["h"][st]), bits(gpu["logits"][st]), sel
+
+
+def _gpu_parity(gpu, W64, hn, xn, sel, K):
+    """The GPU's outputs on the sampled positions against the oracle: top-K
+    (bit-exact), lse (absolute error) and dH rows (max-abs error over the
+    oracle's max-abs), with the bars the tests use."""
+    import numpy as np
+    import oracle
+    T = gpu["h"].shape[0]
+    vals_g = gpu["vals"][sel].cpu().numpy()
+    idx_g = gpu["idx"][sel].cpu().numpy()
+    vals_o, idx_o = oracle.topk_rows(xn, K)
+    topk_exact = bool(np.array_equal(idx_g, idx_o) and
+                      np.array_equal(vals_g.view(np.uint32), vals_o.view(np.uint32)))
+    rows = np.arange(len(sel))
+    lse_o, _ = oracle.forward_rows(hn, W64, vals_o, idx_o, 1.0, rows)
+    lse_err = float(np.abs(gpu["lse"][sel].cpu().numpy().astype(np.float64) - lse_o).max())
+    dH_o = oracle.backward_dH_rows(hn, W64, vals_o, idx_o, 1.0, rows, T)
+    dH_g = gpu["dH"][sel].float().cpu().numpy().astype(np.float64)
+    dH_err = float(np.abs(dH_g - dH_o).max() / max(np.abs(dH_o).max(), 1e-300))
+    return {"rows": int(len(sel)), "topk_bit_exact": topk_exact, "lse_max_abs_err": lse_err,
+            "dH_rel_maxabs_err": dH_err,
+            "bars": {"topk": "bit-exact", "lse_max_abs_err": 1e-3, "dH_rel_maxabs_err": 2e-2},
+            "pass": bool(topk_exact and lse_err <= 1e-3 and dH_err <= 2e-2)}
+
+
+def cpu_baseline(w, rows=0, steps=1, single_core_rows=32, gpu=None):
     """Oracle tokens/s on a bounded sample (rows positions per step), on all
-    host cores and, on a smaller sample, on one core."""
+    host cores and, on a smaller sample, on one core.  Given the bench's device
+    tensors (`gpu`), the sample is rows of the bench's own batch and the GPU's
+    outputs on those rows are checked against the oracle's."""
     if rows <= 0:
         rows = 16
-    W64, hn, xn = _cpu_setup(w, rows)
+    sel = None
+    if gpu is not None:
+        W64, hn, xn, sel = _cpu_from_gpu(gpu, rows)
+        rows = len(sel)
+    else:
+        W64, hn, xn = _cpu_setup(w, rows)
     t0 = time.perf_counter()
     for _ in range(steps):
         _cpu_sample_step(W64, hn, xn, w["K"])
@@ -167,6 +216,10 @@ def cpu_baseline(w, rows=0, steps=1, single_core_rows=32):
             dt1 = time.perf_counter() - t0
         out["single_core"] = {"value": n1 / dt1, "unit": UNIT, "cores": 1,
                               "sample": f"{n1} positions of the same sample; {dt1:.2f} s"}
+    if gpu is not None:
+        out["sample"] = (f"{rows} evenly spaced positions of the bench's own batch (T={w['T']}): "
+                         + out["sample"].split(": ", 1)[1])
+        out["parity"] = _gpu_parity(gpu, W64, hn, xn, sel, w["K"])
     return out
 
 
@@ -304,20 +357,27 @@ def run_kd(args, rank, world):
 
     def step(timing=None, inp=None):
         hh, WW, xx = inp if inp is not None else (h, W, logits)
+        nvtx = torch.cuda.nvtx
         if timing is not None:
             ev_topk[0].record()
+        nvtx.range_push("kd_topk_build")
         st = kd.kd_topk_build(xx.data_ptr(), kd.KD_DTYPE_BF16, T, V, K, vals.data_ptr(),
                               idx.data_ptr(), ws_topk.data_ptr(), ws_topk.numel(), sp)
+        nvtx.range_pop()
         if timing is not None:
             ev_topk[1].record()
+        nvtx.range_push("kd_fused_kl_fwd")
         st |= kd.kd_fused_kl_fwd(hh.data_ptr(), WW.data_ptr(), code, T, d, V, vals.data_ptr(),
                                  idx.data_ptr(), K, chunk, 1.0, loss.data_ptr(), lse.data_ptr(),
                                  None, ws.data_ptr(), ws.numel(), sp)
+        nvtx.range_pop()
         if timing is not None:
             ev_fwd[1].record()
+        nvtx.range_push("kd_fused_kl_bwd")
         st |= kd.kd_fused_kl_bwd(hh.data_ptr(), WW.data_ptr(), code, T, d, V, vals.data_ptr(),
                                  idx.data_ptr(), K, chunk, 1.0, lse.data_ptr(), None, dH.data_ptr(),
                                  dW.data_ptr(), 0, ws.data_ptr(), ws.numel(), sp)
+        nvtx.range_pop()
         if st != 0:
             raise RuntimeError(f"libkd call failed ({st})")
         if timing is not None:
@@ -439,7 +499,10 @@ def run_kd(args, rank, world):
         return
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, rows=args.cpu_rows or 128)
+        torch.cuda.nvtx.range_push("cpu_baseline")
+        cpu = cpu_baseline(w, rows=args.cpu_rows or 128,
+                           gpu=dict(h=h, W=W, logits=logits, vals=vals, idx=idx, lse=lse, dH=dH))
+        torch.cuda.nvtx.range_pop()
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
