@@ -39,12 +39,12 @@ UNIT = "tokens/s"
 # gemm2_step_head-8k-c2048.md), valid only for the GEMM sources with this
 # digest; the roofline's "traffic" is null for any other source.
 NCU_TRAFFIC = {
-    "source_sha256_16": "f75cb9b01e4049e6",
+    "source_sha256_16": "a7dd4ece485234b2",
     # dram__bytes_read.sum + dram__bytes_write.sum per launch of each GEMM kind,
     # from one capture of all 14 GEMM launches of a head-8k-c2048 step (2048-row
     # chunks at d=4096, V=131072: the launch shapes of the 32K head); dW is the
     # mix of a 32K step, one storing and seven accumulating launches
-    "per_launch_bytes": {"fwd_lse": 1.324e9, "bwd_dz": 1.990e9, "dH": 3.690e9, "dW": 6.364e9},
+    "per_launch_bytes": {"fwd_lse": 1.530e9, "bwd_dz": 2.209e9, "dH": 3.975e9, "dW": 6.570e9},
 }
 
 

@@ -17,6 +17,9 @@ ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libkd.so")
+# Same sources with the device-side invariant checks on (-DKD_DEBUG=1): a failed
+# check records KD_ERR_INTERNAL in the workspace's status word.
+DEBUG_LIB_PATH = os.path.join(PKG_DIR, "libkd_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -42,35 +45,39 @@ def deps():
         sorted(glob.glob(os.path.join(CSRC, "*.h"))) + [os.path.join(INCLUDE, "kd.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB_PATH):
+def up_to_date(debug: bool = False) -> bool:
+    lib = DEBUG_LIB_PATH if debug else LIB_PATH
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in deps())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every CUDA source into one shared library; returns its path."""
-    if not force and up_to_date():
-        return LIB_PATH
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile every CUDA source into one shared library; returns its path.
+    ``debug`` builds libkd_debug.so, with the device-side invariant checks."""
+    lib = DEBUG_LIB_PATH if debug else LIB_PATH
+    if not force and up_to_date(debug):
+        return lib
     nvcc = _nvcc()
-    objdir = os.path.join(ROOT, "_build")
+    objdir = os.path.join(ROOT, "_build", "debug" if debug else "")
     os.makedirs(objdir, exist_ok=True)
     objs = []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
-        cmd = [nvcc, *NVCC_FLAGS, "-I" + INCLUDE, "-c", src, "-o", obj]
+        cmd = [nvcc, *NVCC_FLAGS, *(["-DKD_DEBUG=1"] if debug else []), "-I" + INCLUDE, "-c", src,
+               "-o", obj]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
         subprocess.run(cmd, check=True)
         objs.append(obj)
-    tmp = LIB_PATH + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-o", tmp, *objs,
            "-cudart", "static"]
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, debug="--debug" in sys.argv))

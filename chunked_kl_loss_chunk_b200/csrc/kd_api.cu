@@ -69,6 +69,7 @@ const char* kd_status_string(int status) {
     case KD_ERR_BAD_INDEX: return "KD_ERR_BAD_INDEX";
     case KD_ERR_TIMEOUT: return "KD_ERR_TIMEOUT";
     case KD_ERR_CUDA: return "KD_ERR_CUDA";
+    case KD_ERR_INTERNAL: return "KD_ERR_INTERNAL";
     default: return "KD_ERR_UNKNOWN";
   }
 }
@@ -97,7 +98,8 @@ kd_status kd_topk_build(const void* logits, int dtype, int64_t T, int64_t V, int
   const int sms = num_sms_current();
   if (sms <= 0) return KD_ERR_CUDA;
   if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return KD_ERR_CUDA;
-  if (kd::launch_topk_bf16(logits, T, V, K, out_vals, out_idx, s, sms) != cudaSuccess)
+  if (kd::launch_topk_bf16(logits, T, V, K, out_vals, out_idx, static_cast<uint32_t*>(ws), s,
+                           sms) != cudaSuccess)
     return KD_ERR_CUDA;
   return KD_OK;
 }

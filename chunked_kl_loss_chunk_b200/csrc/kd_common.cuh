@@ -23,6 +23,18 @@ __device__ __forceinline__ uint32_t read_status(const uint32_t* status) {
   return *reinterpret_cast<const volatile uint32_t*>(status);
 }
 
+// Invariant checks of the debug build (compiled with -DKD_DEBUG=1, shipped as
+// libkd_debug.so): a failed check records KD_ERR_INTERNAL in the status word
+// (first error wins) and execution goes on; nothing traps.  In the release
+// build the checks compile to nothing.
+#ifndef KD_DEBUG
+#define KD_DEBUG 0
+#endif
+#define KD_CHECK(cond, status)                                              \
+  do {                                                                      \
+    if (KD_DEBUG && !(cond)) ::kd::set_status((status), KD_ERR_INTERNAL);   \
+  } while (0)
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));

@@ -206,6 +206,8 @@ __device__ __forceinline__ void run_epilogue(const GemmArgs& g, const CUtensorMa
           run_m = nm;
         }
       }
+      // every cached index inside this tile's columns was gathered
+      KD_CHECK(!row_ok || static_cast<int64_t>(nidx) >= (n0 + BN < g.V ? n0 + BN : g.V), g.status);
       if (row_ok) g.partials[static_cast<int64_t>(m) * g.n_tiles + nb] =
           make_float4(run_m, run_s, gat, 0.f);
     } else {  // EPI_BWD_DZ: dz box per 32 columns; TMA clips columns >= V, rows >= M
@@ -241,6 +243,7 @@ __device__ __forceinline__ void run_epilogue(const GemmArgs& g, const CUtensorMa
         else stage_box_bf16(box, lane, v);
         emit_box<Elem>(tmC, box, base, y_box, false);
       }
+      KD_CHECK(!row_ok || static_cast<int64_t>(nidx) >= (n0 + BN < g.V ? n0 + BN : g.V), g.status);
     }
   } else {  // EPI_STORE_H (dtype of h), EPI_STORE_PARTIAL (fp32) or EPI_ACCUM_W (fp32)
 #pragma unroll 1

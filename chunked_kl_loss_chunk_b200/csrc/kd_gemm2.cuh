@@ -135,6 +135,7 @@ __device__ __forceinline__ void unit_coords(const GemmArgs& g, int m_tiles2, int
   const int t = u - split * per_split;
   mb2 = g.m_fastest ? t % m_tiles2 : t / g.n_tiles;
   nb = g.m_fastest ? t / m_tiles2 : t % g.n_tiles;
+  KD_CHECK(split < g.k_split && mb2 < m_tiles2 && nb < g.n_tiles, g.status);
 }
 
 // First K block of split s: the k_blocks are divided as evenly as possible,

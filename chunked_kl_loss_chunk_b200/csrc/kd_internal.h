@@ -37,7 +37,7 @@ kd_status fused_bwd(const void* h, const void* W, int dtype, int64_t T, int64_t 
                     int accumulate, void* ws, cudaStream_t s, int num_sms, uint64_t limit_ns);
 
 cudaError_t launch_topk_bf16(const void* logits, int64_t T, int64_t V, int K, float* out_vals,
-                             int32_t* out_idx, cudaStream_t stream, int num_sms);
+                             int32_t* out_idx, uint32_t* status, cudaStream_t stream, int num_sms);
 
 cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
 

@@ -121,6 +121,10 @@ __device__ __forceinline__ void find_bin_256(const uint32_t* h, uint32_t target,
                                              uint32_t* out_above, uint32_t* out_through) {
   if (threadIdx.x >= 32) return;
   const int lane = threadIdx.x;
+  if (KD_DEBUG) {                       // "not found" unless a lane writes a bin below
+    if (lane == 0) *out_bin = 0xFFFFFFFFu;
+    __syncwarp();
+  }
   const uint4 a = reinterpret_cast<const uint4*>(h)[2 * lane];
   const uint4 b = reinterpret_cast<const uint4*>(h)[2 * lane + 1];
   const uint32_t c[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
@@ -299,7 +303,8 @@ __device__ __forceinline__ bool any_ge(__nv_bfloat162 m, __nv_bfloat16 tb) {
 // The row is walked in warp-uniform steps so that every lane takes part in
 // every ballot.
 __device__ __forceinline__ void stream_survivors(TopkSmem& sm, const uint16_t* __restrict__ row,
-                                                 int64_t V, float tf, bool take_all) {
+                                                 int64_t V, float tf, bool take_all,
+                                                 uint32_t* status) {
   const uintptr_t addr = reinterpret_cast<uintptr_t>(row);
   int64_t head = ((16 - (addr & 15)) & 15) >> 1;
   if (head > V) head = V;
@@ -351,6 +356,7 @@ __device__ __forceinline__ void stream_survivors(TopkSmem& sm, const uint16_t* _
         }
         if (pass) {
           const int pos = cnt + __popc(b & lanes_below);
+          KD_CHECK(pos < 32, status);
           sq[pos] = q[u];
           sb[pos] = static_cast<uint32_t>(head + (j << 3));
         }
@@ -367,7 +373,8 @@ __device__ __forceinline__ void stream_survivors(TopkSmem& sm, const uint16_t* _
 
 __global__ void __launch_bounds__(TK_THREADS, 4)
 topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int K,
-                 float* __restrict__ out_vals, int32_t* __restrict__ out_idx) {
+                 float* __restrict__ out_vals, int32_t* __restrict__ out_idx,
+                 uint32_t* __restrict__ status) {
   extern __shared__ __align__(16) unsigned char tk_smem_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_smem_raw);
   const int tid = threadIdx.x;
@@ -433,6 +440,7 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
     // (target <= S: either S == V >= K, or V > 4096 >= 3K)
     find_bin_256(sm.hist, target, &sm.thr_bin, &sm.thr_above, &sm.n_sel);
     __syncthreads();
+    KD_CHECK(sm.thr_bin < 256u, status);
     const uint32_t hb = 255u - sm.thr_bin;            // high byte of L
     const uint32_t above_hb = sm.thr_above;
 #pragma unroll
@@ -442,6 +450,7 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
     __syncthreads();
     find_bin_256(sm.hist + TK_THREADS, target - above_hb, &sm.thr_bin, &sm.thr_above, &sm.n_sel);
     __syncthreads();
+    KD_CHECK(sm.thr_bin < 256u, status);
     const uint32_t L = (hb << 8) | (255u - sm.thr_bin);   // candidate iff order key >= L
     if (tid == 0) sm.n_sel = 0u;
     // Float threshold equivalent on non-NaN values: key >= L <=> x >= tf.
@@ -460,7 +469,7 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
     }
 
     // ---- 2. stream the row, keep survivors ------------------------------------
-    stream_survivors(sm, row, V, tf, take_all);
+    stream_survivors(sm, row, V, tf, take_all, status);
     __syncthreads();
     const uint32_t n = sm.n_cand;
 
@@ -491,6 +500,7 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
         uint32_t* res = sm.warp_tot;                 // scratch: bin, above, through
         find_bin_256(sm.hist, static_cast<uint32_t>(K), &res[0], &res[1], &res[2]);
         __syncthreads();
+        KD_CHECK(res[0] < 256u, status);
         if (tid == 0) {
           sm.thr_bin = L + static_cast<uint32_t>(TK_THREADS - 1) - res[0];   // exact K-th key
           sm.thr_above = res[2];                                            // survivors >= it
@@ -530,7 +540,11 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
       if (compact) {
         for (int i = tid; i < static_cast<int>(n); i += TK_THREADS) {
           const uint64_t c = sm.cand[i];
-          if (comp_key(c) >= Tk) sm.sel[atomicAdd(&sm.n_sel, 1u)] = c;
+          if (comp_key(c) >= Tk) {
+            const uint32_t p = atomicAdd(&sm.n_sel, 1u);
+            KD_CHECK(p < static_cast<uint32_t>(TK_SEL_CAP), status);
+            if (p < static_cast<uint32_t>(TK_SEL_CAP)) sm.sel[p] = c;
+          }
         }
         __syncthreads();
       }
@@ -539,6 +553,7 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
       //     it; those below K write themselves there, already in order.
       const uint64_t* set = compact ? sm.sel : sm.cand;
       const int ns = compact ? static_cast<int>(sm.n_sel) : static_cast<int>(n);
+      KD_CHECK(ns >= K && (!compact || static_cast<uint32_t>(ns) == sm.thr_above), status);
       for (int i = tid; i < ns; i += TK_THREADS) {
         const uint64_t c = set[i];
         int rank = 0;
@@ -576,7 +591,8 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
       const uint32_t b = key >> 4;
       if (b > b1) {
         const uint32_t pos = atomicAdd(&sm.n_sel, 1u);
-        sm.sel[pos] = composite(key, i, bits);
+        KD_CHECK(pos < static_cast<uint32_t>(K), status);
+        if (pos < static_cast<uint32_t>(TK_SEL_CAP)) sm.sel[pos] = composite(key, i, bits);
       } else if (b == b1) {
         atomicAdd(&sm.hist16[key & 15u], 1u);
       }
@@ -610,7 +626,9 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
           const uint32_t key = bf16_order_key(bits);
           if ((key >> 4) == b1 && key > Tk) {
             const uint32_t pos = atomicAdd(&sm.n_sel, 1u);
-            sm.sel[pos] = composite(key, static_cast<uint32_t>(i), bits);
+            KD_CHECK(pos < static_cast<uint32_t>(K), status);
+            if (pos < static_cast<uint32_t>(TK_SEL_CAP))
+              sm.sel[pos] = composite(key, static_cast<uint32_t>(i), bits);
           } else if (key == Tk) {
             eq_mask |= 1u << u;
           }
@@ -625,7 +643,9 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
         if (eq_mask & (1u << u)) {
           if (r < need) {
             const uint32_t pos = atomicAdd(&sm.n_sel, 1u);
-            sm.sel[pos] = composite(Tk, static_cast<uint32_t>(i0 + u), row[i0 + u]);
+            KD_CHECK(pos < static_cast<uint32_t>(K), status);
+            if (pos < static_cast<uint32_t>(TK_SEL_CAP))
+              sm.sel[pos] = composite(Tk, static_cast<uint32_t>(i0 + u), row[i0 + u]);
           }
           ++r;
         }
@@ -634,6 +654,7 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
       if (tid == 0) sm.eq_base = eb + tile_total;
       __syncthreads();
     }
+    KD_CHECK(sm.n_sel == static_cast<uint32_t>(K), status);   // exactly the top K
     const int np = next_pow2(K);
     for (int i = K + tid; i < np; i += TK_THREADS) sm.sel[i] = ~0ull;
     __syncthreads();
@@ -655,7 +676,7 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
 namespace kd {
 
 cudaError_t launch_topk_bf16(const void* logits, int64_t T, int64_t V, int K, float* out_vals,
-                             int32_t* out_idx, cudaStream_t stream, int num_sms) {
+                             int32_t* out_idx, uint32_t* status, cudaStream_t stream, int num_sms) {
   const size_t smem = sizeof(TopkSmem);
   cudaError_t e = cudaFuncSetAttribute(topk_bf16_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -668,7 +689,7 @@ cudaError_t launch_topk_bf16(const void* logits, int64_t T, int64_t V, int K, fl
   int64_t grid = static_cast<int64_t>(num_sms) * per_sm;
   if (grid > T) grid = T;
   topk_bf16_kernel<<<static_cast<unsigned>(grid), TK_THREADS, smem, stream>>>(
-      static_cast<const uint16_t*>(logits), T, V, K, out_vals, out_idx);
+      static_cast<const uint16_t*>(logits), T, V, K, out_vals, out_idx, status);
   count_launch();
   return cudaGetLastError();
 }

@@ -21,10 +21,11 @@ import torch
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG_DIR, "libkd.so")
+DEBUG_LIB_PATH = os.path.join(_PKG_DIR, "libkd_debug.so")   # built with -DKD_DEBUG=1
 HEADER_PATH = os.path.join(os.path.dirname(_PKG_DIR), "include", "kd.h")
 
 KD_OK, KD_ERR_INVALID_ARG, KD_ERR_UNSUPPORTED, KD_ERR_WORKSPACE = 0, 1, 2, 3
-KD_ERR_BAD_INDEX, KD_ERR_TIMEOUT, KD_ERR_CUDA = 4, 5, 6
+KD_ERR_BAD_INDEX, KD_ERR_TIMEOUT, KD_ERR_CUDA, KD_ERR_INTERNAL = 4, 5, 6, 7
 KD_DTYPE_F32, KD_DTYPE_BF16 = 0, 1
 KD_KL_LOGPROB_CACHE, KD_KL_TAU_SQUARED = 0x1, 0x2
 CACHE_KINDS = ("logits", "logprobs")
@@ -86,6 +87,17 @@ def load():
         fn.argtypes = args
     _lib = lib
     return lib
+
+
+def use_library(path: str):
+    """Route every later call to the library at `path` (e.g. DEBUG_LIB_PATH,
+    whose kernels also check internal invariants); returns the previous path."""
+    global _lib, LIB_PATH
+    prev = LIB_PATH
+    LIB_PATH = path
+    _lib = None
+    load()
+    return prev
 
 
 class KDError(RuntimeError):

@@ -43,7 +43,9 @@ typedef enum kd_status {
   KD_ERR_WORKSPACE = 3,    /* ws_bytes smaller than the matching *_workspace_size   */
   KD_ERR_BAD_INDEX = 4,    /* device: a cache index outside [0,V) or repeated in a row */
   KD_ERR_TIMEOUT = 5,      /* device: a pipeline wait exceeded its time limit        */
-  KD_ERR_CUDA = 6          /* a CUDA runtime/driver call failed                      */
+  KD_ERR_CUDA = 6,         /* a CUDA runtime/driver call failed                      */
+  KD_ERR_INTERNAL = 7      /* device: an internal invariant failed (checked only in
+                              the debug build of the library, libkd_debug.so)        */
 } kd_status;
 
 typedef enum kd_dtype {
@@ -181,7 +183,9 @@ kd_status kd_fused_kl_bwd_ex(const void* h, const void* W, int dtype,
                              void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronises `stream`, then returns the device status recorded in `ws`
- * (KD_OK, KD_ERR_BAD_INDEX or KD_ERR_TIMEOUT), or KD_ERR_CUDA. */
+ * (KD_OK, KD_ERR_BAD_INDEX, KD_ERR_TIMEOUT or, in the debug build,
+ * KD_ERR_INTERNAL), or KD_ERR_CUDA.  Works for the workspaces of both
+ * kd_topk_build and the fused loss. */
 kd_status kd_read_device_status(const void* ws, void* stream);
 
 /* ------------------------------------------------------------------------ */

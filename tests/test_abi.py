@@ -32,7 +32,7 @@ def test_every_header_symbol_is_exported(lib):
 def test_status_strings(lib):
     for code, name in [(0, "KD_OK"), (1, "KD_ERR_INVALID_ARG"), (2, "KD_ERR_UNSUPPORTED"),
                        (3, "KD_ERR_WORKSPACE"), (4, "KD_ERR_BAD_INDEX"), (5, "KD_ERR_TIMEOUT"),
-                       (6, "KD_ERR_CUDA")]:
+                       (6, "KD_ERR_CUDA"), (7, "KD_ERR_INTERNAL")]:
         assert kd.status_string(code) == name
     assert kd.status_string(99) == "KD_ERR_UNKNOWN"
     assert kd.load().kd_version() >> 16 == 1
