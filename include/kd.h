@@ -75,6 +75,10 @@ size_t kd_topk_workspace_size(int64_t T, int64_t V, int K);
  *   out_vals float32 [T, K]: exact copies of the selected logits;
  *   out_idx  int32   [T, K]: their column indices.
  * Requires 1 <= K <= min(V, 1024), T >= 1, V < 2^31.
+ * ws (1024-byte aligned, ws_bytes >= kd_topk_workspace_size) holds the
+ * device status word, cleared at the start of the call; only the debug build
+ * records anything there (KD_ERR_INTERNAL).  Read it with
+ * kd_read_device_status.
  */
 kd_status kd_topk_build(const void* logits, int dtype, int64_t T, int64_t V, int K,
                         float* out_vals, int32_t* out_idx,
