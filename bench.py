@@ -66,6 +66,8 @@ def _args():
     ap.add_argument("--workload", default="head-32k")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="time K eager steps instead of K replays of a captured step")
     ap.add_argument("--cpu-rows", type=int, default=0, help="oracle rows per CPU step (0 = auto)")
     ap.add_argument("--sweep-memory", action="store_true",
                     help="print the peak-memory vs T sweep instead of the bench line")
@@ -357,6 +359,7 @@ def run_kd(args, rank, world):
 
     def step(timing=None, inp=None):
         hh, WW, xx = inp if inp is not None else (h, W, logits)
+        sp = torch.cuda.current_stream().cuda_stream     # the capture stream while capturing
         nvtx = torch.cuda.nvtx
         if timing is not None:
             ev_topk[0].record()
@@ -402,7 +405,26 @@ def run_kd(args, rank, world):
     for _ in range(5):
         step(comp)
 
-    prof = kd.GemmProfiler(capacity=4 * ((T + chunk - 1) // chunk) * args.steps + 16)
+    # The timed steps: one step captured in a CUDA graph (the library allocates
+    # nothing and never synchronises inside a call), replayed K times; the
+    # per-GEMM CUDA events are captured with it, so the per-kind figures are
+    # those of the last timed step.  --no-graph times K eager steps instead.
+    per_step_launches = 4 * ((T + chunk - 1) // chunk) + 16
+    prof = kd.GemmProfiler(capacity=per_step_launches * (1 if args.graph else args.steps))
+    graph = None
+    if args.graph:
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(stream)
+        graph = torch.cuda.CUDAGraph()
+        nc = kd.kd_launch_count()
+        with prof:
+            with torch.cuda.graph(graph, stream=side):
+                step()
+        graph_launches = kd.kd_launch_count() - nc
+        stream.wait_stream(side)
+        graph.replay()                                   # upload; untimed
+        torch.cuda.synchronize()
+        assert kd.read_device_status(ws) == kd.KD_OK
     sampler = ClockSampler(local) if rank == 0 else None
     torch.cuda.reset_peak_memory_stats(dev)
     barrier()
@@ -412,13 +434,22 @@ def run_kd(args, rank, world):
         time.sleep(0.3)
     n0 = kd.kd_launch_count()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with prof:
+    if graph is not None:
         e0.record()
         for _ in range(args.steps):
-            step()
+            graph.replay()
         e1.record()
         torch.cuda.synchronize()
-    n_launch = kd.kd_launch_count() - n0
+        n_launch = graph_launches * args.steps            # replays run no host code
+    else:
+        with prof:
+            e0.record()
+            for _ in range(args.steps):
+                step()
+            e1.record()
+            torch.cuda.synchronize()
+        n_launch = kd.kd_launch_count() - n0
+    assert kd.read_device_status(ws) == kd.KD_OK
     clocks = sampler.stop() if sampler else None
     barrier()
     peak_bytes = torch.cuda.max_memory_allocated(dev)
@@ -439,7 +470,8 @@ def run_kd(args, rank, world):
     peaks, peak_src = _peaks()
     peak_sus = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     achieved = dom[1]["flops"] / (dom[1]["ms"] / 1000.0) / 1e12
-    gemm_ms_step = sum(v["ms"] for v in kinds.values()) / args.steps
+    profiled_steps = 1 if graph is not None else args.steps
+    gemm_ms_step = sum(v["ms"] for v in kinds.values()) / profiled_steps
     topk_ms = statistics.median(comp["topk_ms"])
     fwd_ms = statistics.median(comp["fwd_ms"])
     bwd_ms = statistics.median(comp["bwd_ms"])
@@ -509,7 +541,10 @@ def run_kd(args, rank, world):
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
         "data": "synthetic",
-        "config": _config(w, args.workload, {"parallelism": f"replicas x{world}"}),
+        "config": _config(w, args.workload, {
+            "parallelism": f"replicas x{world}",
+            "timed_steps": ("one step captured in a CUDA graph, replayed K times"
+                            if graph is not None else "K eager steps")}),
         "loss_fwd_bwd": {"ms": loss_ms, "tokens_per_s": T / (loss_ms / 1000.0),
                           "tflops": loss_tflops,
                           "frac_bf16_peak_sustained": loss_tflops / peak_sus,

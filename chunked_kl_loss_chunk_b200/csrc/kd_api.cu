@@ -40,10 +40,24 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
 
+// While `s` is being captured into a CUDA graph the record must be external to
+// become an event node of the graph (timed on every replay); outside capture
+// it is a plain record.  A failed record is cleared so that it can never be
+// reported as the failure of the launch it brackets.
+static void record_profile_event(void* ev, cudaStream_t s) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess) cs = cudaStreamCaptureStatusNone;
+  const cudaError_t e =
+      cs == cudaStreamCaptureStatusActive
+          ? cudaEventRecordWithFlags(static_cast<cudaEvent_t>(ev), s, cudaEventRecordExternal)
+          : cudaEventRecord(static_cast<cudaEvent_t>(ev), s);
+  if (e != cudaSuccess) cudaGetLastError();
+}
+
 void profile_before(int kind, double flops, cudaStream_t s) {
   g_prof.armed = false;
   if (!g_prof.start || !(g_prof.mask & kind) || g_prof.n >= g_prof.capacity) return;
-  cudaEventRecord(static_cast<cudaEvent_t>(g_prof.start[g_prof.n]), s);
+  record_profile_event(g_prof.start[g_prof.n], s);
   if (g_prof.kinds) g_prof.kinds[g_prof.n] = kind;
   if (g_prof.flops) g_prof.flops[g_prof.n] = flops;
   g_prof.armed = true;
@@ -51,7 +65,7 @@ void profile_before(int kind, double flops, cudaStream_t s) {
 
 void profile_after(cudaStream_t s) {
   if (!g_prof.armed) return;
-  cudaEventRecord(static_cast<cudaEvent_t>(g_prof.end[g_prof.n]), s);
+  record_profile_event(g_prof.end[g_prof.n], s);
   ++g_prof.n;
   g_prof.armed = false;
 }

@@ -259,7 +259,10 @@ uint64_t kd_launch_count(void);
  * start_events[i] before and end_events[i] after itself on its stream
  * (cudaEvent_t handles created by the caller with timing enabled), and its
  * kind and FLOP count in kinds[i] / flops[i] (host arrays owned by the caller),
- * for i < capacity.  Launches beyond capacity are not recorded. */
+ * for i < capacity.  Launches beyond capacity are not recorded.  The events
+ * are recorded as external records, so launches made while their stream is
+ * being captured into a CUDA graph put event nodes in the graph, timed again
+ * on every replay. */
 kd_status kd_profile_attach(void* const* start_events, void* const* end_events, int* kinds,
                             double* flops, int capacity, int kind_mask);
 
