@@ -413,18 +413,27 @@ def run_kd(args, rank, world):
     prof = kd.GemmProfiler(capacity=per_step_launches * (1 if args.graph else args.steps))
     graph = None
     if args.graph:
-        side = torch.cuda.Stream(device=dev)
-        side.wait_stream(stream)
-        graph = torch.cuda.CUDAGraph()
-        nc = kd.kd_launch_count()
-        with prof:
-            with torch.cuda.graph(graph, stream=side):
-                step()
-        graph_launches = kd.kd_launch_count() - nc
-        stream.wait_stream(side)
-        graph.replay()                                   # upload; untimed
-        torch.cuda.synchronize()
-        assert kd.read_device_status(ws) == kd.KD_OK
+        # thread_local: other threads of the process (e.g. a process group's
+        # watchdog) may keep making CUDA calls while this thread captures
+        try:
+            side = torch.cuda.Stream(device=dev)
+            side.wait_stream(stream)
+            g = torch.cuda.CUDAGraph()
+            nc = kd.kd_launch_count()
+            with prof:
+                with torch.cuda.graph(g, stream=side, capture_error_mode="thread_local"):
+                    step()
+            graph_launches = kd.kd_launch_count() - nc
+            stream.wait_stream(side)
+            g.replay()                                   # upload; untimed
+            torch.cuda.synchronize()
+            assert kd.read_device_status(ws) == kd.KD_OK
+            graph = g
+        except Exception as exc:                         # time eager steps instead
+            print(f"bench: CUDA graph capture failed ({exc!r}); timing eager steps",
+                  file=sys.stderr, flush=True)
+            torch.cuda.synchronize()
+            prof = kd.GemmProfiler(capacity=per_step_launches * args.steps)
     sampler = ClockSampler(local) if rank == 0 else None
     torch.cuda.reset_peak_memory_stats(dev)
     barrier()
