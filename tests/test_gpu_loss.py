@@ -1,7 +1,7 @@
 """GPU parity of the fused chunked KL loss (forward and backward) against the
 fp64 oracle, through the C ABI.
 
-Tolerances (spec bar, written here):
+Tolerances (the parity bar, written here):
   * loss: relative error <= 1e-3;
   * dH, dW: max|gpu - oracle| / max|oracle| <= 2e-2;
   * lse: absolute error <= 1e-3 (bf16 operands multiply exactly and accumulate
