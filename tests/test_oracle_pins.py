@@ -407,6 +407,18 @@ def test_unknown_cache_kind_rejected():
 
 # ---------------------------------------------------------------- inputs
 
+def test_logprob_cache_generator_row_mass():
+    """make_logprob_cache: K log-probabilities per row whose probabilities sum to
+    the drawn row mass S in [0.3, 0.95], the same for every call with a seed."""
+    vals, S = inputs.make_logprob_cache(64, 20, seed=4)
+    assert vals.shape == (64, 20) and vals.dtype == torch.float32 and S.shape == (64,)
+    assert float(S.min()) >= 0.3 and float(S.max()) <= 0.95
+    assert torch.allclose(torch.exp(vals.double()).sum(dim=1), S.double(), rtol=1e-5)
+    assert bool((vals < 0).all())                      # every entry below probability 1
+    v2, S2 = inputs.make_logprob_cache(64, 20, seed=4)
+    assert torch.equal(v2, vals) and torch.equal(S2, S)
+
+
 def test_input_generator_shapes_and_distinct_indices():
     h, W, vals, idx = inputs.make_loss_inputs(64, 32, 500, 16, dtype=torch.float32, seed=0)
     assert h.shape == (64, 32) and W.shape == (500, 32) and vals.shape == (64, 16)
