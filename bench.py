@@ -35,9 +35,9 @@ METRIC = "tokens/s & TFLOP/s (8TdV) fused top-K KL fwd+bwd; % BF16 tensor peak; 
 UNIT = "tokens/s"
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
-# ncu capture of launches shaped exactly like the bench's (profiles/
-# gemm2_step_head-8k-c2048.md), valid only for the GEMM sources with this
-# digest; the roofline's "traffic" is null for any other source.
+# ncu capture of launches shaped exactly like the bench's (a head-8k-c2048 step:
+# 2048-row chunks at d=4096, V=131072), valid only for the GEMM sources with
+# this digest; the roofline's "traffic" is null for any other source.
 NCU_TRAFFIC = {
     "source_sha256_16": "a7dd4ece485234b2",
     # dram__bytes_read.sum + dram__bytes_write.sum per launch of each GEMM kind,

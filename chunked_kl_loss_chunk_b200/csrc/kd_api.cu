@@ -30,7 +30,7 @@ int num_sms_current() {
   return n;
 }
 
-constexpr int KD_MAX_K = 1024;
+using kd::KD_MAX_K;
 
 }  // namespace
 
@@ -68,6 +68,24 @@ void profile_after(cudaStream_t s) {
   record_profile_event(g_prof.end[g_prof.n], s);
   ++g_prof.n;
   g_prof.armed = false;
+}
+
+kd_status validate_loss_inputs(const void* h, const void* W, int dtype, int64_t T, int64_t d,
+                               int64_t V, const float* t_vals, const int32_t* t_idx, int K,
+                               int64_t chunk, float tau) {
+  if (!h || !W || !t_vals || !t_idx) return KD_ERR_INVALID_ARG;
+  if (T < 1 || d < 1 || V < 1 || K < 1 || K > V || chunk < 1) return KD_ERR_INVALID_ARG;
+  if (!(tau > 0.f) || !isfinite(tau)) return KD_ERR_INVALID_ARG;
+  if (!aligned(h, 16) || !aligned(W, 16) || !aligned(t_vals, 16) || !aligned(t_idx, 16))
+    return KD_ERR_INVALID_ARG;
+  if (dtype != KD_DTYPE_BF16 && dtype != KD_DTYPE_F32) return KD_ERR_UNSUPPORTED;
+  if (d % 8 != 0 || K > KD_MAX_K || V >= (int64_t(1) << 31) - 256 ||
+      d >= (int64_t(1) << 31) || T >= (int64_t(1) << 40))
+    return KD_ERR_UNSUPPORTED;
+  // Rows per chunk: the backward contracts dW over two chunks' rows in one
+  // 32-bit GEMM extent.
+  if ((chunk < T ? chunk : T) > (int64_t(1) << 30)) return KD_ERR_UNSUPPORTED;
+  return KD_OK;
 }
 
 }  // namespace kd
@@ -121,26 +139,18 @@ kd_status kd_topk_build(const void* logits, int dtype, int64_t T, int64_t V, int
 size_t kd_fused_kl_workspace_size(int64_t T, int64_t d, int64_t V, int K, int64_t chunk,
                                   int dtype) {
   if (T < 1 || d < 1 || V < 1 || K < 1 || chunk < 1) return 0;
-  return kd::ws_layout(T, d, V, K, chunk, dtype).total;
+  const kd::WsLayout L = kd::ws_layout(T, d, V, K, chunk, dtype);
+  return L.ok ? L.total : 0;
 }
 
 static kd_status validate_loss(const void* h, const void* W, int dtype, int64_t T, int64_t d,
                                int64_t V, const float* t_vals, const int32_t* t_idx, int K,
                                int64_t chunk, float tau, void* ws, size_t ws_bytes) {
-  if (!h || !W || !t_vals || !t_idx || !ws) return KD_ERR_INVALID_ARG;
-  if (T < 1 || d < 1 || V < 1 || K < 1 || K > V || chunk < 1) return KD_ERR_INVALID_ARG;
-  if (!(tau > 0.f) || !isfinite(tau)) return KD_ERR_INVALID_ARG;
-  if (!aligned(h, 16) || !aligned(W, 16) || !aligned(t_vals, 16) || !aligned(t_idx, 16) ||
-      !aligned(ws, 1024))
-    return KD_ERR_INVALID_ARG;
-  if (dtype != KD_DTYPE_BF16 && dtype != KD_DTYPE_F32) return KD_ERR_UNSUPPORTED;
-  if (d % 8 != 0 || K > KD_MAX_K || V >= (int64_t(1) << 31) - 256 ||
-      d >= (int64_t(1) << 31) || T >= (int64_t(1) << 40))
-    return KD_ERR_UNSUPPORTED;
-  // Rows per chunk: the backward contracts dW over two chunks' rows in one
-  // 32-bit GEMM extent.
-  if ((chunk < T ? chunk : T) > (int64_t(1) << 30)) return KD_ERR_UNSUPPORTED;
-  if (ws_bytes < kd::ws_layout(T, d, V, K, chunk, dtype).total) return KD_ERR_WORKSPACE;
+  const kd_status st = kd::validate_loss_inputs(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, tau);
+  if (st != KD_OK) return st;
+  if (!ws || !aligned(ws, kd::KD_WS_ALIGN)) return KD_ERR_INVALID_ARG;
+  const kd::WsLayout L = kd::ws_layout(T, d, V, K, chunk, dtype);
+  if (!L.ok || ws_bytes < L.total) return KD_ERR_WORKSPACE;
   return KD_OK;
 }
 

@@ -17,14 +17,38 @@ constexpr int KD_DH_MAX_SPLIT = 4;
 // updated once per group (its read-modify-write traffic falls by this factor).
 constexpr int KD_DW_GROUP = 2;
 
+// Largest number of cached teacher entries per position (the prep kernel
+// sorts a row's entries in shared memory, and the top-K build keeps up to this
+// many in its selection buffer).
+constexpr int KD_MAX_K = 1024;
+
+// Alignment of every region of a fused-loss workspace, and of its base: the
+// tensor maps encoded over the dz scratch and the dH partials need at least
+// 16 bytes, and the regions are placed at multiples of this.
+constexpr size_t KD_WS_ALIGN = 1024;
+
 // Byte offsets of the regions of a fused-loss workspace.
+// Every size is computed with overflow checks: when a byte count does not fit
+// in size_t, `ok` is false and every offset from that point on, and `total`,
+// read SIZE_MAX, so no finite workspace is ever accepted for such sizes.
 struct WsLayout {
   size_t p_sorted = 0, idx_sorted = 0, stats = 0, kl = 0, scratch = 0, hpart = 0, total = 0;
+  size_t fwd_end = 0;    // end of the forward's partials (the forward uses nothing beyond)
   int64_t ldz = 0;       // row pitch (elements) of the dz scratch
   int64_t rows_pad = 0;  // chunk rows rounded up to 256 (rows per dH partial)
+  bool ok = true;
 };
 
 WsLayout ws_layout(int64_t T, int64_t d, int64_t V, int K, int64_t chunk, int dtype);
+
+// Host validation shared by every fused-loss entry point, for everything but
+// the workspace and the outputs: non-null, 16-byte-aligned inputs; positive
+// sizes with K <= V; a finite tau > 0 (KD_ERR_INVALID_ARG); a supported dtype,
+// d % 8 == 0, K <= KD_MAX_K, V < 2^31 - 256, d < 2^31, T < 2^40 and
+// min(chunk, T) <= 2^30 (KD_ERR_UNSUPPORTED).  Makes no CUDA call.
+kd_status validate_loss_inputs(const void* h, const void* W, int dtype, int64_t T, int64_t d,
+                               int64_t V, const float* t_vals, const int32_t* t_idx, int K,
+                               int64_t chunk, float tau);
 
 kd_status fused_fwd(const void* h, const void* W, int dtype, int64_t T, int64_t d, int64_t V,
                     const float* t_vals, const int32_t* t_idx, int K, int64_t chunk, float tau,

@@ -34,7 +34,7 @@ static inline double loss_weight(float tau, uint32_t flags) {
 // moved past V.
 // ----------------------------------------------------------------------------
 constexpr int PREP_WARPS = 4;
-constexpr int PREP_MAXK = 1024;
+constexpr int PREP_MAXK = KD_MAX_K;
 
 __global__ void __launch_bounds__(PREP_WARPS * 32)
 prep_kernel(const float* __restrict__ vals, const int32_t* __restrict__ idx, int64_t T, int K,
@@ -368,31 +368,63 @@ inline int cdiv(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b)
 
 }  // namespace
 
+namespace {
+
+// size_t arithmetic that saturates at SIZE_MAX and clears `ok` on overflow.
+struct CheckedSize {
+  bool ok = true;
+  size_t mul(size_t a, size_t b) {
+    size_t r;
+    if (!ok || __builtin_mul_overflow(a, b, &r)) return fail();
+    return r;
+  }
+  size_t add(size_t a, size_t b) {
+    size_t r;
+    if (!ok || __builtin_add_overflow(a, b, &r)) return fail();
+    return r;
+  }
+  size_t align(size_t x) {   // round up to KD_WS_ALIGN
+    const size_t r = add(x, KD_WS_ALIGN - 1);
+    return ok ? (r & ~(KD_WS_ALIGN - 1)) : r;
+  }
+  size_t fail() {
+    ok = false;
+    return SIZE_MAX;
+  }
+};
+
+}  // namespace
+
 WsLayout ws_layout(int64_t T, int64_t d, int64_t V, int K, int64_t chunk, int dtype) {
   WsLayout L;
+  CheckedSize c;
   const size_t es = dtype == KD_DTYPE_F32 ? 4 : 2;
-  auto al = [](size_t x) { return (x + 1023) & ~static_cast<size_t>(1023); };
-  size_t off = 1024;  // status word + reserved
+  const size_t t = static_cast<size_t>(T), k = static_cast<size_t>(K);
+  size_t off = KD_WS_ALIGN;  // status word + reserved
   L.p_sorted = off;
-  off = al(off + static_cast<size_t>(T) * K * 4);
+  off = c.align(c.add(off, c.mul(c.mul(t, k), 4)));
   L.idx_sorted = off;
-  off = al(off + static_cast<size_t>(T) * K * 4);
+  off = c.align(c.add(off, c.mul(c.mul(t, k), 4)));
   L.stats = off;
-  off = al(off + static_cast<size_t>(T) * 8);
+  off = c.align(c.add(off, c.mul(t, 8)));
   L.kl = off;
-  off = al(off + static_cast<size_t>(T) * 4);
+  off = c.align(c.add(off, c.mul(t, 4)));
   const int64_t rows = chunk < T ? chunk : T;
   L.ldz = ((V + 63) / 64) * 64;
   const size_t n_tiles = static_cast<size_t>((V + BN - 1) / BN);
-  const size_t part = static_cast<size_t>(rows) * n_tiles * 16;
-  const size_t dz =
-      static_cast<size_t>(KD_DW_GROUP) * static_cast<size_t>(rows) * static_cast<size_t>(L.ldz) * es;
+  const size_t part = c.mul(c.mul(static_cast<size_t>(rows), n_tiles), 16);
+  const size_t dz = c.mul(c.mul(c.mul(KD_DW_GROUP, static_cast<size_t>(rows)),
+                                static_cast<size_t>(L.ldz)), es);
   L.scratch = off;
-  off = al(off + (part > dz ? part : dz));
+  L.fwd_end = c.add(off, part);
+  off = c.align(c.add(off, part > dz ? part : dz));
   L.rows_pad = ((rows + 255) / 256) * 256;
   L.hpart = off;
-  off = al(off + static_cast<size_t>(KD_DH_MAX_SPLIT) * L.rows_pad * static_cast<size_t>(d) * 4);
+  off = c.align(c.add(off, c.mul(c.mul(KD_DH_MAX_SPLIT, static_cast<size_t>(L.rows_pad)),
+                                 c.mul(static_cast<size_t>(d), 4))));
   L.total = off;
+  L.ok = c.ok;
+  if (!L.ok) L.total = L.fwd_end = SIZE_MAX;
   return L;
 }
 

@@ -29,6 +29,7 @@ constexpr int TK_BINS = 4096;       // bins of (order key >> 4)
 constexpr int TK_SAMPLE = 4096;
 constexpr int TK_CAND_CAP = 2048;
 constexpr int TK_SEL_CAP = 1024;    // >= K
+static_assert(TK_SEL_CAP >= KD_MAX_K, "the selection buffer holds every K the ABI accepts");
 constexpr int TK_UNROLL = 8;        // 16-byte loads in flight per thread
 constexpr int SAMPLE_PER_THREAD = TK_SAMPLE / TK_THREADS;   // 16
 

@@ -222,16 +222,22 @@ kd_status kd_debug_wait_probe(void* ws, size_t ws_bytes, uint64_t limit_ns, void
  * cannot provide a workspace -- for example a plugin that receives only its
  * input and output pointers, or a program whose device memory all belongs to
  * another framework's pool.  Scratch comes from a fixed array inside the
- * library; nothing is allocated.
+ * library (1024-byte aligned, like a caller workspace); nothing is allocated.
+ *   - The arguments are checked exactly as kd_fused_kl_fwd checks them (same
+ *     ranges and status codes) before anything else happens.
  *   - Scratch needed: about 8*T*K + 12*T + 16*min(chunk,T)*ceil(V/256) bytes
- *     plus alignment; when that exceeds KD_NOALLOC_SCRATCH_BYTES the call
- *     returns KD_ERR_WORKSPACE and launches nothing (e.g. T=32768, K=100,
- *     chunk=2048, V=131072 needs about 43 MB and fits).
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
- *   - All calls share the one array: calls that can overlap on the GPU (other
- *     streams, other threads) race and give wrong results; serialise them.
+ *     plus alignment, computed with overflow checks; when that exceeds
+ *     KD_NOALLOC_SCRATCH_BYTES the call returns KD_ERR_WORKSPACE and launches
+ *     nothing (e.g. T=32768, K=100, chunk=2048, V=131072 needs about 43 MB and
+ *     fits).
+ *   - The first call in a CUDA context looks up the array's device address in
+ *     that context (cudaGetSymbolAddress, with the device current) and caches
+ *     it under the context's unique id; make that first call before any stream
+ *     capture.
+ *   - All calls on a device share the one array, which keeps the last call's
+ *     contents (each call rewrites every part it reads): calls that can
+ *     overlap on the GPU (other streams, other threads) race and give wrong
+ *     results; serialise them.
  *   - Device-side status (bad cache index, timeout) goes to the array's status
  *     word, which this ABI does not expose; use kd_fused_kl_fwd with a
  *     workspace when that check matters.

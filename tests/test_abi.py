@@ -191,3 +191,56 @@ def test_missing_library_fails_loudly(monkeypatch):
     monkeypatch.setattr(kd, "LIB_PATH", "/nonexistent/libkd.so")
     with pytest.raises(RuntimeError):
         kd.load()
+
+
+def _fwd_noalloc(**kw):
+    a = dict(h=FAKE, W=FAKE, dtype=kd.KD_DTYPE_BF16, T=256, d=256, V=4096, vals=FAKE, idx=FAKE,
+             K=16, chunk=64, tau=1.0, loss=FAKE, lse=FAKE, kl=None, stream=None)
+    a.update(kw)
+    return kd.kd_fused_kl_fwd_noalloc(a["h"], a["W"], a["dtype"], a["T"], a["d"], a["V"], a["vals"],
+                                      a["idx"], a["K"], a["chunk"], a["tau"], a["loss"], a["lse"],
+                                      a["kl"], a["stream"])
+
+
+def test_noalloc_validation_matches_the_workspace_forward(lib):
+    """The entry point without a workspace checks its arguments with the same
+    routine as kd_fused_kl_fwd: same ranges, same status codes, before any CUDA
+    call (so these run without a GPU)."""
+    for kw, want in [
+        (dict(h=None), kd.KD_ERR_INVALID_ARG),
+        (dict(lse=None), kd.KD_ERR_INVALID_ARG),
+        (dict(loss=None), kd.KD_ERR_INVALID_ARG),
+        (dict(T=0), kd.KD_ERR_INVALID_ARG),
+        (dict(K=4097), kd.KD_ERR_INVALID_ARG),
+        (dict(tau=float("nan")), kd.KD_ERR_INVALID_ARG),
+        (dict(h=FAKE + 8), kd.KD_ERR_INVALID_ARG),
+        (dict(kl=FAKE + 4), kd.KD_ERR_INVALID_ARG),
+        (dict(dtype=7), kd.KD_ERR_UNSUPPORTED),
+        (dict(d=12), kd.KD_ERR_UNSUPPORTED),
+        (dict(K=1025), kd.KD_ERR_UNSUPPORTED),
+        (dict(V=(1 << 31) - 200), kd.KD_ERR_UNSUPPORTED),
+        (dict(T=1 << 40), kd.KD_ERR_UNSUPPORTED),
+        (dict(T=1 << 62, K=4), kd.KD_ERR_UNSUPPORTED),   # T*K*4 etc. would wrap in size_t
+        (dict(T=1 << 31, chunk=1 << 31), kd.KD_ERR_UNSUPPORTED),  # chunk rows above 2^30
+    ]:
+        assert _fwd_noalloc(**kw) == want, kw
+        if "kl" not in kw and "loss" not in kw and "lse" not in kw:
+            assert _fwd(**{k: v for k, v in kw.items()}) == want, kw
+
+
+def test_noalloc_rejects_what_does_not_fit(lib):
+    # 2^20 positions x K=100: 800 MB of sorted cache, far above the 64 MiB array
+    assert _fwd_noalloc(T=1 << 20, K=100, V=131072) == kd.KD_ERR_WORKSPACE
+    # the largest T under 2^40 with K = 1024 still needs more than the array
+    assert _fwd_noalloc(T=(1 << 40) - 1, K=1024, V=131072) == kd.KD_ERR_WORKSPACE
+
+
+def test_workspace_size_reports_zero_when_it_cannot_be_represented(lib):
+    # four fp32 dH partials of 2^30 chunk rows x d ~ 2^31: 2^65 bytes
+    d = (1 << 31) - 8
+    assert kd.kd_fused_kl_workspace_size(1 << 30, d, 4096, 1, 1 << 30, kd.KD_DTYPE_F32) == 0
+    # and the fused calls reject that size with KD_ERR_WORKSPACE, never a wrapped size
+    assert _fwd(T=1 << 30, d=d, V=4096, K=1, chunk=1 << 30, dtype=kd.KD_DTYPE_F32,
+                ws_bytes=(1 << 64) - 1) == kd.KD_ERR_WORKSPACE
+    assert _bwd(T=1 << 30, d=d, V=4096, K=1, chunk=1 << 30, dtype=kd.KD_DTYPE_F32,
+                ws_bytes=(1 << 64) - 1) == kd.KD_ERR_WORKSPACE
