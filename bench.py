@@ -69,6 +69,8 @@ def _args():
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time K eager steps instead of K replays of a captured step")
     ap.add_argument("--cpu-rows", type=int, default=0, help="oracle rows per CPU step (0 = auto)")
+    ap.add_argument("--no-topk-alone", action="store_true",
+                    help="skip timing the top-K build on its own after the timed steps")
     ap.add_argument("--sweep-memory", action="store_true",
                     help="print the peak-memory vs T sweep instead of the bench line")
     return ap.parse_args()
@@ -353,46 +355,64 @@ def run_kd(args, rank, world):
     stream = torch.cuda.current_stream()
     sp = stream.cuda_stream
     code = kd.KD_DTYPE_BF16 if dt == torch.bfloat16 else kd.KD_DTYPE_F32
-    ev_topk = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    ev_fwd = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    ev_bwd = torch.cuda.Event(enable_timing=True)
 
-    def step(timing=None, inp=None):
+    def step(ev=None, inp=None):
+        """One step; `ev` (4 timing events) marks its start and the ends of the
+        top-K build, the forward and the backward on the launching stream."""
         hh, WW, xx = inp if inp is not None else (h, W, logits)
         sp = torch.cuda.current_stream().cuda_stream     # the capture stream while capturing
         nvtx = torch.cuda.nvtx
-        if timing is not None:
-            ev_topk[0].record()
+        if ev is not None:
+            ev[0].record()
         nvtx.range_push("kd_topk_build")
         st = kd.kd_topk_build(xx.data_ptr(), kd.KD_DTYPE_BF16, T, V, K, vals.data_ptr(),
                               idx.data_ptr(), ws_topk.data_ptr(), ws_topk.numel(), sp)
         nvtx.range_pop()
-        if timing is not None:
-            ev_topk[1].record()
+        if ev is not None:
+            ev[1].record()
         nvtx.range_push("kd_fused_kl_fwd")
         st |= kd.kd_fused_kl_fwd(hh.data_ptr(), WW.data_ptr(), code, T, d, V, vals.data_ptr(),
                                  idx.data_ptr(), K, chunk, 1.0, loss.data_ptr(), lse.data_ptr(),
                                  None, ws.data_ptr(), ws.numel(), sp)
         nvtx.range_pop()
-        if timing is not None:
-            ev_fwd[1].record()
+        if ev is not None:
+            ev[2].record()
         nvtx.range_push("kd_fused_kl_bwd")
         st |= kd.kd_fused_kl_bwd(hh.data_ptr(), WW.data_ptr(), code, T, d, V, vals.data_ptr(),
                                  idx.data_ptr(), K, chunk, 1.0, lse.data_ptr(), None, dH.data_ptr(),
                                  dW.data_ptr(), 0, ws.data_ptr(), ws.numel(), sp)
         nvtx.range_pop()
+        if ev is not None:
+            ev[3].record()
         if st != 0:
             raise RuntimeError(f"libkd call failed ({st})")
-        if timing is not None:
-            ev_bwd.record()
-            torch.cuda.synchronize()
-            timing["topk_ms"].append(ev_topk[0].elapsed_time(ev_topk[1]))
-            timing["fwd_ms"].append(ev_topk[1].elapsed_time(ev_fwd[1]))
-            timing["bwd_ms"].append(ev_fwd[1].elapsed_time(ev_bwd))
 
     def barrier():
         if world > 1:
             dist.barrier()
+
+    def capture(fn, n_launch_out):
+        """Capture fn() into a CUDA graph on a side stream; returns the graph,
+        or None (after printing why) when capture fails."""
+        try:
+            side = torch.cuda.Stream(device=dev)
+            side.wait_stream(stream)
+            g = torch.cuda.CUDAGraph()
+            nc = kd.kd_launch_count()
+            # thread_local: other threads of the process (e.g. a process group's
+            # watchdog) may keep making CUDA calls while this thread captures
+            with torch.cuda.graph(g, stream=side, capture_error_mode="thread_local"):
+                fn()
+            n_launch_out.append(kd.kd_launch_count() - nc)
+            stream.wait_stream(side)
+            g.replay()                                   # upload; untimed
+            torch.cuda.synchronize()
+            return g
+        except Exception as exc:
+            print(f"bench: CUDA graph capture failed ({exc!r}); timing eager steps",
+                  file=sys.stderr, flush=True)
+            torch.cuda.synchronize()
+            return None
 
     # warm-up
     for _ in range(args.warmup):
@@ -400,40 +420,26 @@ def run_kd(args, rank, world):
     torch.cuda.synchronize()
     assert kd.read_device_status(ws) == kd.KD_OK
 
-    # component timings (separate passes outside the timed region; medians)
-    comp = {"topk_ms": [], "fwd_ms": [], "bwd_ms": []}
-    for _ in range(5):
-        step(comp)
-
-    # The timed steps: one step captured in a CUDA graph (the library allocates
-    # nothing and never synchronises inside a call), replayed K times; the
-    # per-GEMM CUDA events are captured with it, so the per-kind figures are
-    # those of the last timed step.  --no-graph times K eager steps instead.
+    # The timed region: K steps captured, one after the other, in ONE CUDA graph
+    # (the library allocates nothing and never synchronises inside a call) and
+    # run by one replay.  Each step carries its own four timing events and
+    # every GEMM launch its own pair (external event nodes of the graph), so
+    # the top-K, forward and backward times, and the per-GEMM figures, are
+    # those of the K timed steps themselves.  --no-graph times K eager steps,
+    # with the same events.
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+           for _ in range(args.steps)]
     per_step_launches = 4 * ((T + chunk - 1) // chunk) + 16
-    prof = kd.GemmProfiler(capacity=per_step_launches * (1 if args.graph else args.steps))
+    prof = kd.GemmProfiler(capacity=per_step_launches * args.steps)
     graph = None
+    graph_launches = []
     if args.graph:
-        # thread_local: other threads of the process (e.g. a process group's
-        # watchdog) may keep making CUDA calls while this thread captures
-        try:
-            side = torch.cuda.Stream(device=dev)
-            side.wait_stream(stream)
-            g = torch.cuda.CUDAGraph()
-            nc = kd.kd_launch_count()
-            with prof:
-                with torch.cuda.graph(g, stream=side, capture_error_mode="thread_local"):
-                    step()
-            graph_launches = kd.kd_launch_count() - nc
-            stream.wait_stream(side)
-            g.replay()                                   # upload; untimed
-            torch.cuda.synchronize()
-            assert kd.read_device_status(ws) == kd.KD_OK
-            graph = g
-        except Exception as exc:                         # time eager steps instead
-            print(f"bench: CUDA graph capture failed ({exc!r}); timing eager steps",
-                  file=sys.stderr, flush=True)
-            torch.cuda.synchronize()
+        with prof:
+            graph = capture(lambda: [step(evs[i]) for i in range(args.steps)], graph_launches)
+        if graph is None:
             prof = kd.GemmProfiler(capacity=per_step_launches * args.steps)
+        else:
+            assert kd.read_device_status(ws) == kd.KD_OK
     sampler = ClockSampler(local) if rank == 0 else None
     torch.cuda.reset_peak_memory_stats(dev)
     barrier()
@@ -445,16 +451,15 @@ def run_kd(args, rank, world):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if graph is not None:
         e0.record()
-        for _ in range(args.steps):
-            graph.replay()
+        graph.replay()
         e1.record()
         torch.cuda.synchronize()
-        n_launch = graph_launches * args.steps            # replays run no host code
+        n_launch = graph_launches[0]                      # a replay runs no host code
     else:
         with prof:
             e0.record()
-            for _ in range(args.steps):
-                step()
+            for i in range(args.steps):
+                step(evs[i])
             e1.record()
             torch.cuda.synchronize()
         n_launch = kd.kd_launch_count() - n0
@@ -464,8 +469,17 @@ def run_kd(args, rank, world):
     peak_bytes = torch.cuda.max_memory_allocated(dev)
     ms_total, value = job_throughput(e0.elapsed_time(e1), T * args.steps, world, dev)
     ms_step = ms_total / args.steps
-    tokens = T * args.steps * world
     flop_step = 8.0 * T * d * V
+
+    # components of the timed steps (sums over the K steps, per step below)
+    topk_sum = sum(e[0].elapsed_time(e[1]) for e in evs)
+    fwd_sum = sum(e[1].elapsed_time(e[2]) for e in evs)
+    bwd_sum = sum(e[2].elapsed_time(e[3]) for e in evs)
+    gaps_sum = sum(evs[i][3].elapsed_time(evs[i + 1][0]) for i in range(args.steps - 1))
+    local_region_ms = e0.elapsed_time(e1)
+    topk_ms = topk_sum / args.steps
+    fwd_ms = fwd_sum / args.steps
+    bwd_ms = bwd_sum / args.steps
 
     # per-GEMM-kind breakdown from the live events
     res = prof.results()
@@ -479,13 +493,47 @@ def run_kd(args, rank, world):
     peaks, peak_src = _peaks()
     peak_sus = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
     achieved = dom[1]["flops"] / (dom[1]["ms"] / 1000.0) / 1e12
-    profiled_steps = 1 if graph is not None else args.steps
-    gemm_ms_step = sum(v["ms"] for v in kinds.values()) / profiled_steps
-    topk_ms = statistics.median(comp["topk_ms"])
-    fwd_ms = statistics.median(comp["fwd_ms"])
-    bwd_ms = statistics.median(comp["bwd_ms"])
-    loss_ms = ms_step - topk_ms
+    gemm_ms_step = sum(v["ms"] for v in kinds.values()) / args.steps
+    loss_ms = fwd_ms + bwd_ms
     loss_tflops = flop_step / (loss_ms / 1000.0) / 1e12
+    topk_bytes = T * V * 2 + T * K * 8
+
+    # The top-K build timed alone: R builds in one graph, clocks sampled, after
+    # the timed region (so it is not part of the step's number).
+    topk_alone = None
+    if rank == 0 and not args.no_topk_alone:
+        R = 20
+        ev_a = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+
+        def topk_only():
+            sp_ = torch.cuda.current_stream().cuda_stream
+            ev_a[0].record()
+            for _ in range(R):
+                st_ = kd.kd_topk_build(logits.data_ptr(), kd.KD_DTYPE_BF16, T, V, K,
+                                       vals.data_ptr(), idx.data_ptr(), ws_topk.data_ptr(),
+                                       ws_topk.numel(), sp_)
+                if st_ != 0:
+                    raise RuntimeError(f"kd_topk_build failed ({st_})")
+            ev_a[1].record()
+        gt = capture(topk_only, []) if args.graph else None
+        samp = ClockSampler(local)
+        torch.cuda.synchronize()
+        samp.start()
+        time.sleep(0.3)
+        for _ in range(3):
+            if gt is not None:
+                gt.replay()
+            else:
+                topk_only()
+        torch.cuda.synchronize()
+        ck = samp.stop()
+        assert kd.read_device_status(ws_topk) == kd.KD_OK
+        ms_a = ev_a[0].elapsed_time(ev_a[1]) / R           # the last replay's R builds
+        topk_alone = {"ms": ms_a, "gbs": topk_bytes / (ms_a / 1000.0) / 1e9,
+                      "frac_hbm_peak": topk_bytes / (ms_a / 1000.0) / 1e9 / float(peaks["hbm_gbs"]),
+                      "builds": R, "clocks": ck,
+                      "note": "the same build timed alone, back to back, outside the step"}
+        del gt
 
     # loss-path memory: what the fused loss holds (inputs, cache, outputs, workspace)
     loss_path_bytes = (h.numel() * h.element_size() + W.numel() * W.element_size()
@@ -552,7 +600,7 @@ def run_kd(args, rank, world):
         "data": "synthetic",
         "config": _config(w, args.workload, {
             "parallelism": f"replicas x{world}",
-            "timed_steps": ("one step captured in a CUDA graph, replayed K times"
+            "timed_steps": ("K steps captured in one CUDA graph, run by one replay"
                             if graph is not None else "K eager steps")}),
         "loss_fwd_bwd": {"ms": loss_ms, "tokens_per_s": T / (loss_ms / 1000.0),
                           "tflops": loss_tflops,
@@ -560,9 +608,17 @@ def run_kd(args, rank, world):
                           "frac_bf16_peak_burst": loss_tflops / float(peaks["bf16_tflops"]),
                           "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
                           "gemm_ms": gemm_ms_step},
-        "topk_build": {"ms": topk_ms, "gbs": (T * V * 2 + T * K * 8) / (topk_ms / 1000.0) / 1e9,
-                       "frac_hbm_peak": (T * V * 2 + T * K * 8) / (topk_ms / 1000.0) / 1e9
-                       / float(peaks["hbm_gbs"])},
+        "topk_build": {"ms": topk_ms, "gbs": topk_bytes / (topk_ms / 1000.0) / 1e9,
+                       "frac_hbm_peak": topk_bytes / (topk_ms / 1000.0) / 1e9
+                       / float(peaks["hbm_gbs"]),
+                       "bytes": int(topk_bytes)},
+        "topk_build_alone": topk_alone,
+        "components": {
+            "source": "CUDA events of the timed steps (inside the timed region)",
+            "topk_ms": topk_ms, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+            "between_steps_ms": gaps_sum / args.steps,
+            "sum_over_ms_per_step": (topk_sum + fwd_sum + bwd_sum + gaps_sum)
+            / max(local_region_ms, 1e-9)},
         "gemm_kernels": {k: {"launches": v["launches"], "ms_per_launch": v["ms"] / v["launches"],
                              "tflops": v["flops"] / (v["ms"] / 1000.0) / 1e12}
                          for k, v in kinds.items()},

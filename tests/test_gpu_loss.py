@@ -334,6 +334,53 @@ def test_dW_sampled_vocab_rows_full_width():
     assert abs(r["loss"].item() - loss_o) <= LOSS_RTOL * abs(loss_o)
 
 
+def _dW_rows_parity_accumulating(T, d, V, K, chunk, tail_rows=0, n_random=32, seed=0):
+    """dW element by element on sampled vocabulary rows, at full d and V, over a
+    backward whose dW launches mostly ADD into dW (one launch per group of two
+    chunks: the first stores, every later one reduce-adds).  The reference is
+    the oracle's own: it computes LSE_t of every position itself (one full fp64
+    projection) and never reads the GPU's lse.  The rows checked are 0, V-1,
+    every teacher index of three positions (one in the first group, one in a
+    middle group, the last position), random rows and, optionally, the last
+    `tail_rows` rows (the ragged last M tile of the dW GEMM when V % 256 != 0).
+    A lost, doubled or stored-instead-of-added group changes every one of them."""
+    groups = -(-T // (2 * chunk))
+    assert groups >= 3, "the check wants at least two accumulating dW launches"
+    r = _run(T, d, V, K, chunk, torch.bfloat16, seed=seed)
+    hn, Wn = to_np_exact(r["h"]), to_np_exact(r["W"])
+    vals, idx = r["vals"].cpu().numpy(), r["idx"].cpu().numpy()
+    rng = np.random.default_rng(seed + 7)
+    pos = [0, T // 2 + 1, T - 1]
+    vrows = np.unique(np.concatenate([idx[pos].ravel(), rng.choice(V, n_random, replace=False),
+                                      [0, V - 1], np.arange(V - tail_rows, V)]).astype(np.int64))
+    dW_o = oracle.backward_dW_rows(hn, Wn, vals, idx, 1.0, vrows)
+    dW_g = r["dW"][torch.as_tensor(vrows, device="cuda")].cpu().numpy()
+    err = rel_maxabs(dW_g, dW_o)
+    assert err <= GRAD_TOL, err
+    # every checked row is non-trivial (a zeroed row would fail the bar above)
+    assert np.abs(dW_o).max(axis=1).min() > 0.0
+    return err
+
+
+@pytest.mark.slow
+def test_dW_full_size_head_8k_accumulating():
+    """T=8192, d=4096, V=131072, K=100, chunk=1024: four dW launches, three of
+    them reduce-adding into dW."""
+    require_gpu()
+    cfg = inputs.WORKLOADS["head-8k"]
+    _dW_rows_parity_accumulating(cfg["T"], cfg["d"], cfg["V"], cfg["K"], cfg["chunk"])
+
+
+@pytest.mark.slow
+def test_dW_full_size_large_vocab_accumulating():
+    """d=2880, V=201088 (V % 256 = 128), K=100, chunk=1024, T=6144: three dW
+    launches, two of them reduce-adding, and the last 128 vocabulary rows (the
+    ragged M tail of every dW launch) checked element by element."""
+    require_gpu()
+    cfg = inputs.WORKLOADS["vocab-201k"]
+    _dW_rows_parity_accumulating(6144, cfg["d"], cfg["V"], cfg["K"], 1024, tail_rows=128)
+
+
 @pytest.mark.slow
 def test_peak_memory_linear_in_T():
     """Peak device memory of fwd + bwd grows linearly in T (the pages: memory
