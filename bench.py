@@ -69,6 +69,9 @@ def _args():
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time K eager steps instead of K replays of a captured step")
     ap.add_argument("--cpu-rows", type=int, default=0, help="oracle rows per CPU step (0 = auto)")
+    ap.add_argument("--dp", action="store_true",
+                    help="data-parallel shards: each rank's T rows are one shard of a batch of "
+                         "T x N positions; dW and the loss are summed over the ranks (NCCL)")
     ap.add_argument("--no-topk-alone", action="store_true",
                     help="skip timing the top-K build on its own after the timed steps")
     ap.add_argument("--sweep-memory", action="store_true",
@@ -348,7 +351,8 @@ def run_kd(args, rank, world):
     idx = torch.empty((T, K), dtype=torch.int32, device=dev)
     ws_topk = kd.alloc_workspace(kd.kd_topk_workspace_size(T, V, K), dev)
     ws = kd.workspace_for(h, W, K, chunk)
-    loss = torch.empty((), dtype=torch.float32, device=dev)
+    loss_vec = torch.empty((1,), dtype=torch.float32, device=dev)
+    loss = loss_vec[0]
     lse = torch.empty((T,), dtype=torch.float32, device=dev)
     dH = torch.empty_like(h)
     dW = torch.empty((V, d), dtype=torch.float32, device=dev)
@@ -371,17 +375,33 @@ def run_kd(args, rank, world):
         if ev is not None:
             ev[1].record()
         nvtx.range_push("kd_fused_kl_fwd")
-        st |= kd.kd_fused_kl_fwd(hh.data_ptr(), WW.data_ptr(), code, T, d, V, vals.data_ptr(),
-                                 idx.data_ptr(), K, chunk, 1.0, loss.data_ptr(), lse.data_ptr(),
-                                 None, ws.data_ptr(), ws.numel(), sp)
+        if args.dp:     # this rank's rows are one shard of a batch of T * world positions
+            st |= kd.kd_fused_kl_fwd_shard(hh.data_ptr(), WW.data_ptr(), code, T, d, V,
+                                           vals.data_ptr(), idx.data_ptr(), K, chunk, 1.0, 0,
+                                           T * world, loss.data_ptr(), lse.data_ptr(), None,
+                                           ws.data_ptr(), ws.numel(), sp)
+        else:
+            st |= kd.kd_fused_kl_fwd(hh.data_ptr(), WW.data_ptr(), code, T, d, V, vals.data_ptr(),
+                                     idx.data_ptr(), K, chunk, 1.0, loss.data_ptr(), lse.data_ptr(),
+                                     None, ws.data_ptr(), ws.numel(), sp)
         nvtx.range_pop()
         if ev is not None:
             ev[2].record()
         nvtx.range_push("kd_fused_kl_bwd")
-        st |= kd.kd_fused_kl_bwd(hh.data_ptr(), WW.data_ptr(), code, T, d, V, vals.data_ptr(),
-                                 idx.data_ptr(), K, chunk, 1.0, lse.data_ptr(), None, dH.data_ptr(),
-                                 dW.data_ptr(), 0, ws.data_ptr(), ws.numel(), sp)
+        if args.dp:
+            st |= kd.kd_fused_kl_bwd_shard(hh.data_ptr(), WW.data_ptr(), code, T, d, V,
+                                           vals.data_ptr(), idx.data_ptr(), K, chunk, 1.0, 0,
+                                           T * world, lse.data_ptr(), None, dH.data_ptr(),
+                                           dW.data_ptr(), 0, ws.data_ptr(), ws.numel(), sp)
+        else:
+            st |= kd.kd_fused_kl_bwd(hh.data_ptr(), WW.data_ptr(), code, T, d, V, vals.data_ptr(),
+                                     idx.data_ptr(), K, chunk, 1.0, lse.data_ptr(), None,
+                                     dH.data_ptr(), dW.data_ptr(), 0, ws.data_ptr(), ws.numel(), sp)
         nvtx.range_pop()
+        if args.dp and world > 1:
+            # the batch's dW and loss: one sum over the ranks (NCCL)
+            dist.all_reduce(dW, op=dist.ReduceOp.SUM)
+            dist.all_reduce(loss_vec, op=dist.ReduceOp.SUM)
         if ev is not None:
             ev[3].record()
         if st != 0:
@@ -433,6 +453,9 @@ def run_kd(args, rank, world):
     prof = kd.GemmProfiler(capacity=per_step_launches * args.steps)
     graph = None
     graph_launches = []
+    if args.dp and world > 1 and args.graph:
+        # the step holds NCCL collectives: time eager steps rather than capture them
+        args.graph = False
     if args.graph:
         with prof:
             graph = capture(lambda: [step(evs[i]) for i in range(args.steps)], graph_launches)
@@ -599,7 +622,8 @@ def run_kd(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if dt == torch.bfloat16 else "f32",
         "data": "synthetic",
         "config": _config(w, args.workload, {
-            "parallelism": f"replicas x{world}",
+            "parallelism": (f"dp{world} (T-sharded batch of {T * world} positions, "
+                            "all-reduce of dW and the loss)" if args.dp else f"replicas x{world}"),
             "timed_steps": ("K steps captured in one CUDA graph, run by one replay"
                             if graph is not None else "K eager steps")}),
         "loss_fwd_bwd": {"ms": loss_ms, "tokens_per_s": T / (loss_ms / 1000.0),

@@ -154,30 +154,79 @@ static kd_status validate_loss(const void* h, const void* W, int dtype, int64_t 
   return KD_OK;
 }
 
-kd_status kd_fused_kl_fwd_ex(const void* h, const void* W, int dtype, int64_t T, int64_t d,
-                             int64_t V, const float* t_vals, const int32_t* t_idx, int K,
-                             int64_t chunk, float temperature, uint32_t flags, float* loss,
-                             float* lse, float* kl_rows, void* ws, size_t ws_bytes,
-                             void* stream) {
+}  // extern "C"
+
+// The forward and backward behind every fused-loss entry point; T_norm is the
+// count the loss and gradients are normalised by (T, or a whole batch's
+// positions for a data-parallel shard of it).
+static kd_status fwd_entry(const void* h, const void* W, int dtype, int64_t T, int64_t T_norm,
+                           int64_t d, int64_t V, const float* t_vals, const int32_t* t_idx,
+                           int K, int64_t chunk, float temperature, uint32_t flags, float* loss,
+                           float* lse, float* kl_rows, void* ws, size_t ws_bytes, void* stream) {
   kd_status st =
       validate_loss(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, ws, ws_bytes);
   if (st != KD_OK) return st;
   if ((flags & ~KD_KL_KNOWN_FLAGS) != 0u) return KD_ERR_INVALID_ARG;
+  if (T_norm < T) return KD_ERR_INVALID_ARG;
+  if (T_norm >= (int64_t(1) << 40)) return KD_ERR_UNSUPPORTED;
   if (!loss || !lse) return KD_ERR_INVALID_ARG;
   if (!aligned(loss, 4) || !aligned(lse, 16) || (kl_rows && !aligned(kl_rows, 16)))
     return KD_ERR_INVALID_ARG;
   const int sms = num_sms_current();
   if (sms <= 0) return KD_ERR_CUDA;
-  return kd::fused_fwd(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, flags, loss,
-                       lse, kl_rows, ws, static_cast<cudaStream_t>(stream), sms, kd::wait_limit_ns());
+  return kd::fused_fwd(h, W, dtype, T, T_norm, d, V, t_vals, t_idx, K, chunk, temperature, flags,
+                       loss, lse, kl_rows, ws, static_cast<cudaStream_t>(stream), sms,
+                       kd::wait_limit_ns());
+}
+
+static kd_status bwd_entry(const void* h, const void* W, int dtype, int64_t T, int64_t T_norm,
+                           int64_t d, int64_t V, const float* t_vals, const int32_t* t_idx,
+                           int K, int64_t chunk, float temperature, uint32_t flags,
+                           const float* lse, const float* grad_loss, void* dH, float* dW,
+                           int accumulate_dW, void* ws, size_t ws_bytes, void* stream) {
+  kd_status st =
+      validate_loss(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, ws, ws_bytes);
+  if (st != KD_OK) return st;
+  if ((flags & ~KD_KL_KNOWN_FLAGS) != 0u) return KD_ERR_INVALID_ARG;
+  if (T_norm < T) return KD_ERR_INVALID_ARG;
+  if (T_norm >= (int64_t(1) << 40)) return KD_ERR_UNSUPPORTED;
+  if (!lse || !dH || !dW) return KD_ERR_INVALID_ARG;
+  if (!aligned(lse, 16) || !aligned(dH, 16) || !aligned(dW, 16) ||
+      (grad_loss && !aligned(grad_loss, 4)))
+    return KD_ERR_INVALID_ARG;
+  const int sms = num_sms_current();
+  if (sms <= 0) return KD_ERR_CUDA;
+  return kd::fused_bwd(h, W, dtype, T, T_norm, d, V, t_vals, t_idx, K, chunk, temperature, flags,
+                       lse, grad_loss, dH, dW, accumulate_dW, ws,
+                       static_cast<cudaStream_t>(stream), sms, kd::wait_limit_ns());
+}
+
+extern "C" {
+
+kd_status kd_fused_kl_fwd_ex(const void* h, const void* W, int dtype, int64_t T, int64_t d,
+                             int64_t V, const float* t_vals, const int32_t* t_idx, int K,
+                             int64_t chunk, float temperature, uint32_t flags, float* loss,
+                             float* lse, float* kl_rows, void* ws, size_t ws_bytes,
+                             void* stream) {
+  return fwd_entry(h, W, dtype, T, T, d, V, t_vals, t_idx, K, chunk, temperature, flags, loss, lse,
+                   kl_rows, ws, ws_bytes, stream);
 }
 
 kd_status kd_fused_kl_fwd(const void* h, const void* W, int dtype, int64_t T, int64_t d,
                           int64_t V, const float* t_vals, const int32_t* t_idx, int K,
                           int64_t chunk, float temperature, float* loss, float* lse,
                           float* kl_rows, void* ws, size_t ws_bytes, void* stream) {
-  return kd_fused_kl_fwd_ex(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, 0u, loss,
-                            lse, kl_rows, ws, ws_bytes, stream);
+  return fwd_entry(h, W, dtype, T, T, d, V, t_vals, t_idx, K, chunk, temperature, 0u, loss, lse,
+                   kl_rows, ws, ws_bytes, stream);
+}
+
+kd_status kd_fused_kl_fwd_shard(const void* h, const void* W, int dtype, int64_t T, int64_t d,
+                                int64_t V, const float* t_vals, const int32_t* t_idx, int K,
+                                int64_t chunk, float temperature, uint32_t flags, int64_t T_total,
+                                float* loss, float* lse, float* kl_rows, void* ws,
+                                size_t ws_bytes, void* stream) {
+  return fwd_entry(h, W, dtype, T, T_total, d, V, t_vals, t_idx, K, chunk, temperature, flags,
+                   loss, lse, kl_rows, ws, ws_bytes, stream);
 }
 
 kd_status kd_fused_kl_bwd_ex(const void* h, const void* W, int dtype, int64_t T, int64_t d,
@@ -185,19 +234,8 @@ kd_status kd_fused_kl_bwd_ex(const void* h, const void* W, int dtype, int64_t T,
                              int64_t chunk, float temperature, uint32_t flags, const float* lse,
                              const float* grad_loss, void* dH, float* dW, int accumulate_dW,
                              void* ws, size_t ws_bytes, void* stream) {
-  kd_status st =
-      validate_loss(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, ws, ws_bytes);
-  if (st != KD_OK) return st;
-  if ((flags & ~KD_KL_KNOWN_FLAGS) != 0u) return KD_ERR_INVALID_ARG;
-  if (!lse || !dH || !dW) return KD_ERR_INVALID_ARG;
-  if (!aligned(lse, 16) || !aligned(dH, 16) || !aligned(dW, 16) ||
-      (grad_loss && !aligned(grad_loss, 4)))
-    return KD_ERR_INVALID_ARG;
-  const int sms = num_sms_current();
-  if (sms <= 0) return KD_ERR_CUDA;
-  return kd::fused_bwd(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, flags, lse,
-                       grad_loss, dH, dW, accumulate_dW, ws, static_cast<cudaStream_t>(stream),
-                       sms, kd::wait_limit_ns());
+  return bwd_entry(h, W, dtype, T, T, d, V, t_vals, t_idx, K, chunk, temperature, flags, lse,
+                   grad_loss, dH, dW, accumulate_dW, ws, ws_bytes, stream);
 }
 
 kd_status kd_fused_kl_bwd(const void* h, const void* W, int dtype, int64_t T, int64_t d,
@@ -205,8 +243,17 @@ kd_status kd_fused_kl_bwd(const void* h, const void* W, int dtype, int64_t T, in
                           int64_t chunk, float temperature, const float* lse,
                           const float* grad_loss, void* dH, float* dW, int accumulate_dW,
                           void* ws, size_t ws_bytes, void* stream) {
-  return kd_fused_kl_bwd_ex(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, 0u, lse,
-                            grad_loss, dH, dW, accumulate_dW, ws, ws_bytes, stream);
+  return bwd_entry(h, W, dtype, T, T, d, V, t_vals, t_idx, K, chunk, temperature, 0u, lse,
+                   grad_loss, dH, dW, accumulate_dW, ws, ws_bytes, stream);
+}
+
+kd_status kd_fused_kl_bwd_shard(const void* h, const void* W, int dtype, int64_t T, int64_t d,
+                                int64_t V, const float* t_vals, const int32_t* t_idx, int K,
+                                int64_t chunk, float temperature, uint32_t flags, int64_t T_total,
+                                const float* lse, const float* grad_loss, void* dH, float* dW,
+                                int accumulate_dW, void* ws, size_t ws_bytes, void* stream) {
+  return bwd_entry(h, W, dtype, T, T_total, d, V, t_vals, t_idx, K, chunk, temperature, flags, lse,
+                   grad_loss, dH, dW, accumulate_dW, ws, ws_bytes, stream);
 }
 
 kd_status kd_read_device_status(const void* ws, void* stream) {

@@ -50,15 +50,20 @@ kd_status validate_loss_inputs(const void* h, const void* W, int dtype, int64_t 
                                int64_t V, const float* t_vals, const int32_t* t_idx, int K,
                                int64_t chunk, float tau);
 
-kd_status fused_fwd(const void* h, const void* W, int dtype, int64_t T, int64_t d, int64_t V,
-                    const float* t_vals, const int32_t* t_idx, int K, int64_t chunk, float tau,
-                    uint32_t flags, float* loss, float* lse, float* kl_rows, void* ws, cudaStream_t s,
-                    int num_sms, uint64_t limit_ns);
+// The fused loss over T positions whose loss and gradients are normalised by
+// T_norm >= T: T_norm == T for a whole batch, the batch's total positions when
+// these T rows are one data-parallel shard of it (then the shards' losses and
+// dW contributions sum to the batch's).
+kd_status fused_fwd(const void* h, const void* W, int dtype, int64_t T, int64_t T_norm, int64_t d,
+                    int64_t V, const float* t_vals, const int32_t* t_idx, int K, int64_t chunk,
+                    float tau, uint32_t flags, float* loss, float* lse, float* kl_rows, void* ws,
+                    cudaStream_t s, int num_sms, uint64_t limit_ns);
 
-kd_status fused_bwd(const void* h, const void* W, int dtype, int64_t T, int64_t d, int64_t V,
-                    const float* t_vals, const int32_t* t_idx, int K, int64_t chunk, float tau,
-                    uint32_t flags, const float* lse, const float* grad_loss, void* dH, float* dW,
-                    int accumulate, void* ws, cudaStream_t s, int num_sms, uint64_t limit_ns);
+kd_status fused_bwd(const void* h, const void* W, int dtype, int64_t T, int64_t T_norm, int64_t d,
+                    int64_t V, const float* t_vals, const int32_t* t_idx, int K, int64_t chunk,
+                    float tau, uint32_t flags, const float* lse, const float* grad_loss, void* dH,
+                    float* dW, int accumulate, void* ws, cudaStream_t s, int num_sms,
+                    uint64_t limit_ns);
 
 cudaError_t launch_topk_bf16(const void* logits, int64_t T, int64_t V, int K, float* out_vals,
                              int32_t* out_idx, uint32_t* status, cudaStream_t stream, int num_sms);

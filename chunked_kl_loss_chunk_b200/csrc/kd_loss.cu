@@ -199,10 +199,12 @@ dh_reduce_kernel(const float* __restrict__ part, int k_split, int64_t split_rows
   }
 }
 
-// Deterministic mean of kl[0..T): one block, fixed per-thread strides, fixed
-// tree; fp64 accumulation.
+// Deterministic sum of kl[0..T) divided by T_norm (T itself, or the positions
+// of the whole batch when these T rows are one data-parallel shard of it): one
+// block, fixed per-thread strides, fixed tree; fp64 accumulation.
 __global__ void __launch_bounds__(1024)
-mean_kernel(const float* __restrict__ kl, int64_t T, double scale, float* __restrict__ loss) {
+mean_kernel(const float* __restrict__ kl, int64_t T, int64_t T_norm, double scale,
+            float* __restrict__ loss) {
   __shared__ double part[1024];
   double acc = 0.0;
   for (int64_t i = threadIdx.x; i < T; i += 1024) acc += static_cast<double>(kl[i]);
@@ -212,7 +214,7 @@ mean_kernel(const float* __restrict__ kl, int64_t T, double scale, float* __rest
     if (threadIdx.x < s) part[threadIdx.x] += part[threadIdx.x + s];
     __syncthreads();
   }
-  if (threadIdx.x == 0) *loss = static_cast<float>(scale * (part[0] / static_cast<double>(T)));
+  if (threadIdx.x == 0) *loss = static_cast<float>(scale * (part[0] / static_cast<double>(T_norm)));
 }
 
 // Failure-detection probe: waits on a barrier that nothing arrives at.
@@ -429,10 +431,11 @@ WsLayout ws_layout(int64_t T, int64_t d, int64_t V, int K, int64_t chunk, int dt
 }
 
 template <typename Elem>
-static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t d, int64_t V,
-                          const float* t_vals, const int32_t* t_idx, int K, int64_t chunk,
-                          float tau, uint32_t flags, float* loss, float* lse, float* kl_rows,
-                          void* ws, cudaStream_t s, int num_sms, uint64_t limit_ns) {
+static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t T_norm, int64_t d,
+                          int64_t V, const float* t_vals, const int32_t* t_idx, int K,
+                          int64_t chunk, float tau, uint32_t flags, float* loss, float* lse,
+                          float* kl_rows, void* ws, cudaStream_t s, int num_sms,
+                          uint64_t limit_ns) {
   constexpr bool F32 = sizeof(Elem) == 4;
   constexpr int BK = ElemCfg<Elem>::BK;
   const WsLayout L = ws_layout(T, d, V, K, chunk, F32 ? KD_DTYPE_F32 : KD_DTYPE_BF16);
@@ -492,18 +495,18 @@ static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
     count_launch();
     if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
   }
-  mean_kernel<<<1, 1024, 0, s>>>(kl, T, loss_weight(tau, flags), loss);
+  mean_kernel<<<1, 1024, 0, s>>>(kl, T, T_norm, loss_weight(tau, flags), loss);
   count_launch();
   if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
   return KD_OK;
 }
 
 template <typename Elem>
-static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, int64_t V,
-                          const float* t_vals, const int32_t* t_idx, int K, int64_t chunk,
-                          float tau, uint32_t flags, const float* lse, const float* grad_loss,
-                          void* dH, float* dW, int accumulate, void* ws, cudaStream_t s,
-                          int num_sms, uint64_t limit_ns) {
+static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t T_norm, int64_t d,
+                          int64_t V, const float* t_vals, const int32_t* t_idx, int K,
+                          int64_t chunk, float tau, uint32_t flags, const float* lse,
+                          const float* grad_loss, void* dH, float* dW, int accumulate, void* ws,
+                          cudaStream_t s, int num_sms, uint64_t limit_ns) {
   constexpr bool F32 = sizeof(Elem) == 4;
   constexpr int BK = ElemCfg<Elem>::BK;
   constexpr int INNER = ROW_BYTES / sizeof(Elem);
@@ -535,7 +538,7 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
   if (!make_out_map(&tHP_out, hpart, true, d, KD_DH_MAX_SPLIT * L.rows_pad, d)) return KD_ERR_CUDA;
   const float zscale = 1.4426950408889634f * inv_tau;
   const float inv_T_tau =
-      static_cast<float>(loss_weight(tau, flags) / (static_cast<double>(T) * tau));
+      static_cast<float>(loss_weight(tau, flags) / (static_cast<double>(T_norm) * tau));
   // dz of KD_DW_GROUP consecutive chunks is kept side by side, so that dW is
   // updated once per group with K = the group's rows (halving dW's
   // read-modify-write traffic); dz and dH are formed chunk by chunk.
@@ -641,26 +644,26 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t d, in
   return KD_OK;
 }
 
-kd_status fused_fwd(const void* h, const void* W, int dtype, int64_t T, int64_t d, int64_t V,
-                    const float* t_vals, const int32_t* t_idx, int K, int64_t chunk, float tau,
-                    uint32_t flags, float* loss, float* lse, float* kl_rows, void* ws,
+kd_status fused_fwd(const void* h, const void* W, int dtype, int64_t T, int64_t T_norm, int64_t d,
+                    int64_t V, const float* t_vals, const int32_t* t_idx, int K, int64_t chunk,
+                    float tau, uint32_t flags, float* loss, float* lse, float* kl_rows, void* ws,
                     cudaStream_t s, int num_sms, uint64_t limit_ns) {
   if (dtype == KD_DTYPE_F32)
-    return fwd_impl<float>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, flags, loss, lse,
+    return fwd_impl<float>(h, W, T, T_norm, d, V, t_vals, t_idx, K, chunk, tau, flags, loss, lse,
                            kl_rows, ws, s, num_sms, limit_ns);
-  return fwd_impl<__nv_bfloat16>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, flags, loss, lse,
-                                 kl_rows, ws, s, num_sms, limit_ns);
+  return fwd_impl<__nv_bfloat16>(h, W, T, T_norm, d, V, t_vals, t_idx, K, chunk, tau, flags, loss,
+                                 lse, kl_rows, ws, s, num_sms, limit_ns);
 }
 
-kd_status fused_bwd(const void* h, const void* W, int dtype, int64_t T, int64_t d, int64_t V,
-                    const float* t_vals, const int32_t* t_idx, int K, int64_t chunk, float tau,
-                    uint32_t flags, const float* lse, const float* grad_loss, void* dH,
+kd_status fused_bwd(const void* h, const void* W, int dtype, int64_t T, int64_t T_norm, int64_t d,
+                    int64_t V, const float* t_vals, const int32_t* t_idx, int K, int64_t chunk,
+                    float tau, uint32_t flags, const float* lse, const float* grad_loss, void* dH,
                     float* dW, int accumulate, void* ws, cudaStream_t s, int num_sms,
                     uint64_t limit_ns) {
   if (dtype == KD_DTYPE_F32)
-    return bwd_impl<float>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, flags, lse, grad_loss,
-                           dH, dW, accumulate, ws, s, num_sms, limit_ns);
-  return bwd_impl<__nv_bfloat16>(h, W, T, d, V, t_vals, t_idx, K, chunk, tau, flags, lse,
+    return bwd_impl<float>(h, W, T, T_norm, d, V, t_vals, t_idx, K, chunk, tau, flags, lse,
+                           grad_loss, dH, dW, accumulate, ws, s, num_sms, limit_ns);
+  return bwd_impl<__nv_bfloat16>(h, W, T, T_norm, d, V, t_vals, t_idx, K, chunk, tau, flags, lse,
                                  grad_loss, dH, dW, accumulate, ws, s, num_sms, limit_ns);
 }
 

@@ -119,7 +119,7 @@ extern "C" kd_status kd_fused_kl_fwd_noalloc(const void* h, const void* W, int d
   // fused_fwd clears the status word itself and overwrites every other region
   // it reads before reading it, so nothing left by a previous call leaks into
   // this one.
-  return kd::fused_fwd(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, 0u, loss,
+  return kd::fused_fwd(h, W, dtype, T, T, d, V, t_vals, t_idx, K, chunk, temperature, 0u, loss,
                        lse, kl_rows, ws, static_cast<cudaStream_t>(stream), sms,
                        kd::wait_limit_ns());
 }

@@ -50,6 +50,12 @@ _SIGNATURES = {
     "kd_fused_kl_bwd_ex": (_c_int, [_c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp, _c_int,
                                     _c_i64, ctypes.c_float, _c_u32, _c_vp, _c_vp, _c_vp, _c_vp, _c_int,
                                     _c_vp, _c_sz, _c_vp]),
+    "kd_fused_kl_fwd_shard": (_c_int, [_c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp,
+                                       _c_int, _c_i64, ctypes.c_float, _c_u32, _c_i64, _c_vp, _c_vp,
+                                       _c_vp, _c_vp, _c_sz, _c_vp]),
+    "kd_fused_kl_bwd_shard": (_c_int, [_c_vp, _c_vp, _c_int, _c_i64, _c_i64, _c_i64, _c_vp, _c_vp,
+                                       _c_int, _c_i64, ctypes.c_float, _c_u32, _c_i64, _c_vp, _c_vp,
+                                       _c_vp, _c_vp, _c_int, _c_vp, _c_sz, _c_vp]),
     "kd_read_device_status": (_c_int, [_c_vp, _c_vp]),
     "kd_set_wait_limit_ns": (_c_int, [_c_u64]),
     "kd_debug_wait_probe": (_c_int, [_c_vp, _c_sz, _c_u64, _c_vp]),
@@ -152,6 +158,19 @@ def kd_fused_kl_bwd_ex(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperatur
     return load().kd_fused_kl_bwd_ex(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature,
                                      flags, lse, grad_loss, dH, dW, accumulate_dW, ws, ws_bytes,
                                      stream)
+
+
+def kd_fused_kl_fwd_shard(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, flags,
+                          T_total, loss, lse, kl_rows, ws, ws_bytes, stream):
+    return load().kd_fused_kl_fwd_shard(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature,
+                                        flags, T_total, loss, lse, kl_rows, ws, ws_bytes, stream)
+
+
+def kd_fused_kl_bwd_shard(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, flags,
+                          T_total, lse, grad_loss, dH, dW, accumulate_dW, ws, ws_bytes, stream):
+    return load().kd_fused_kl_bwd_shard(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature,
+                                        flags, T_total, lse, grad_loss, dH, dW, accumulate_dW, ws,
+                                        ws_bytes, stream)
 
 
 def kd_fused_kl_fwd_noalloc(h, W, dtype, T, d, V, t_vals, t_idx, K, chunk, temperature, loss, lse,
@@ -284,8 +303,11 @@ def kl_flags(cache: str = "logits", tau_squared: bool = False) -> int:
 
 def fused_kl_fwd(h, W, t_vals, t_idx, chunk: int, temperature: float = 1.0, ws=None,
                  kl_rows: bool = False, stream=None, cache: str = "logits",
-                 tau_squared: bool = False):
-    """Returns (loss [] f32, lse [T] f32, kl [T] f32 or None, ws)."""
+                 tau_squared: bool = False, T_total: int | None = None):
+    """Returns (loss [] f32, lse [T] f32, kl [T] f32 or None, ws).  With
+    ``T_total`` the rows are one data-parallel shard of a batch of T_total
+    positions (kd_fused_kl_fwd_shard): the loss is this shard's part of the
+    batch's mean."""
     for t in (h, W, t_vals, t_idx):
         assert t.is_cuda and t.is_contiguous()
     T, d = h.shape
@@ -297,18 +319,29 @@ def fused_kl_fwd(h, W, t_vals, t_idx, chunk: int, temperature: float = 1.0, ws=N
     loss = torch.empty((), dtype=torch.float32, device=h.device)
     lse = torch.empty((T,), dtype=torch.float32, device=h.device)
     kl = torch.empty((T,), dtype=torch.float32, device=h.device) if kl_rows else None
-    _check(kd_fused_kl_fwd_ex(h.data_ptr(), W.data_ptr(), _dtype_code(h), T, d, V,
-                              t_vals.data_ptr(), t_idx.data_ptr(), K, chunk, float(temperature),
-                              flags, loss.data_ptr(), lse.data_ptr(), _ptr(kl), ws.data_ptr(),
-                              ws.numel(), _stream(stream)),
-           "kd_fused_kl_fwd_ex")
+    if T_total is None:
+        _check(kd_fused_kl_fwd_ex(h.data_ptr(), W.data_ptr(), _dtype_code(h), T, d, V,
+                                  t_vals.data_ptr(), t_idx.data_ptr(), K, chunk, float(temperature),
+                                  flags, loss.data_ptr(), lse.data_ptr(), _ptr(kl), ws.data_ptr(),
+                                  ws.numel(), _stream(stream)),
+               "kd_fused_kl_fwd_ex")
+    else:
+        _check(kd_fused_kl_fwd_shard(h.data_ptr(), W.data_ptr(), _dtype_code(h), T, d, V,
+                                     t_vals.data_ptr(), t_idx.data_ptr(), K, chunk,
+                                     float(temperature), flags, int(T_total), loss.data_ptr(),
+                                     lse.data_ptr(), _ptr(kl), ws.data_ptr(), ws.numel(),
+                                     _stream(stream)),
+               "kd_fused_kl_fwd_shard")
     return loss, lse, kl, ws
 
 
 def fused_kl_bwd(h, W, t_vals, t_idx, lse, chunk: int, temperature: float = 1.0, grad_loss=None,
                  ws=None, dH=None, dW=None, accumulate_dW: bool = False, stream=None,
-                 cache: str = "logits", tau_squared: bool = False):
-    """Returns (dH [T,d] dtype of h, dW [V,d] f32, ws)."""
+                 cache: str = "logits", tau_squared: bool = False, T_total: int | None = None):
+    """Returns (dH [T,d] dtype of h, dW [V,d] f32, ws).  With ``T_total`` the
+    rows are one data-parallel shard of a batch of T_total positions
+    (kd_fused_kl_bwd_shard): dH is the batch gradient's rows of this shard and
+    dW this shard's term of the batch's dW."""
     T, d = h.shape
     V = W.shape[0]
     K = t_vals.shape[1]
@@ -319,11 +352,21 @@ def fused_kl_bwd(h, W, t_vals, t_idx, lse, chunk: int, temperature: float = 1.0,
         dH = torch.empty_like(h)
     if dW is None:
         dW = torch.empty((V, d), dtype=torch.float32, device=h.device)
-    _check(kd_fused_kl_bwd_ex(h.data_ptr(), W.data_ptr(), _dtype_code(h), T, d, V,
-                              t_vals.data_ptr(), t_idx.data_ptr(), K, chunk, float(temperature),
-                              flags, lse.data_ptr(), _ptr(grad_loss), dH.data_ptr(), dW.data_ptr(),
-                              int(accumulate_dW), ws.data_ptr(), ws.numel(), _stream(stream)),
-           "kd_fused_kl_bwd_ex")
+    if T_total is None:
+        _check(kd_fused_kl_bwd_ex(h.data_ptr(), W.data_ptr(), _dtype_code(h), T, d, V,
+                                  t_vals.data_ptr(), t_idx.data_ptr(), K, chunk, float(temperature),
+                                  flags, lse.data_ptr(), _ptr(grad_loss), dH.data_ptr(),
+                                  dW.data_ptr(), int(accumulate_dW), ws.data_ptr(), ws.numel(),
+                                  _stream(stream)),
+               "kd_fused_kl_bwd_ex")
+    else:
+        _check(kd_fused_kl_bwd_shard(h.data_ptr(), W.data_ptr(), _dtype_code(h), T, d, V,
+                                     t_vals.data_ptr(), t_idx.data_ptr(), K, chunk,
+                                     float(temperature), flags, int(T_total), lse.data_ptr(),
+                                     _ptr(grad_loss), dH.data_ptr(), dW.data_ptr(),
+                                     int(accumulate_dW), ws.data_ptr(), ws.numel(),
+                                     _stream(stream)),
+               "kd_fused_kl_bwd_shard")
     return dH, dW, ws
 
 

@@ -186,6 +186,49 @@ kd_status kd_fused_kl_bwd_ex(const void* h, const void* W, int dtype,
                              void* dH, float* dW, int accumulate_dW,
                              void* ws, size_t ws_bytes, void* stream);
 
+/* ------------------------------------------------------------------------ */
+/* Data-parallel shards.  The loss is a mean over positions and every       */
+/* position's terms are independent, so a batch of T_total positions can be */
+/* split along T over ranks: each rank runs the fused loss on its own rows  */
+/* and only the scalar loss and dW (a sum over positions) are summed across */
+/* ranks afterwards (an all-reduce; the pages' method runs on one GPU --    */
+/* [GX] "Detailed Chronology and Technical Evolution" and [AS] "What a      */
+/* Single H200 GPU Can Now Do That Once Required Four Nodes" describe the   */
+/* multi-GPU sharding it replaces).                                          */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * kd_fused_kl_fwd_ex / kd_fused_kl_bwd_ex for T rows that are one shard of a
+ * batch of T_total >= T positions: every 1/T of the plain calls becomes
+ * 1/T_total.
+ *   loss  = (1/T_total) sum over this shard's rows of KL_t (times tau^2 under
+ *           KD_KL_TAU_SQUARED), so the shards' losses sum to the batch's loss;
+ *   dz_tv = g / (T_total tau) * (...), so dH holds exactly the batch gradient's
+ *           rows of this shard and dW this shard's term of the batch's dW (the
+ *           sum of the shards' dW is the batch's dW; accumulate_dW may chain
+ *           shards on one device).
+ * lse and kl_rows are per position and do not depend on T_total.  With
+ * T_total == T these are the _ex calls, bit for bit.  T_total < T returns
+ * KD_ERR_INVALID_ARG; T_total >= 2^40 returns KD_ERR_UNSUPPORTED.  The
+ * workspace is sized for the shard: kd_fused_kl_workspace_size(T, ...).
+ */
+kd_status kd_fused_kl_fwd_shard(const void* h, const void* W, int dtype,
+                                int64_t T, int64_t d, int64_t V,
+                                const float* t_vals, const int32_t* t_idx, int K,
+                                int64_t chunk, float temperature, uint32_t flags,
+                                int64_t T_total,
+                                float* loss, float* lse, float* kl_rows,
+                                void* ws, size_t ws_bytes, void* stream);
+
+kd_status kd_fused_kl_bwd_shard(const void* h, const void* W, int dtype,
+                                int64_t T, int64_t d, int64_t V,
+                                const float* t_vals, const int32_t* t_idx, int K,
+                                int64_t chunk, float temperature, uint32_t flags,
+                                int64_t T_total,
+                                const float* lse, const float* grad_loss,
+                                void* dH, float* dW, int accumulate_dW,
+                                void* ws, size_t ws_bytes, void* stream);
+
 /* Synchronises `stream`, then returns the device status recorded in `ws`
  * (KD_OK, KD_ERR_BAD_INDEX, KD_ERR_TIMEOUT or, in the debug build,
  * KD_ERR_INTERNAL), or KD_ERR_CUDA.  Works for the workspaces of both

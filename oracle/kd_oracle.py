@@ -174,9 +174,13 @@ def _kl_from(a_rows, lse_rows, p_rows, idx_rows):
 # ---------------------------------------------------------------------------
 
 def forward(h, W, vals, idx, tau: float = 1.0, row_block: int = 256, cache: str = "logits",
-            tau_sq: bool = False):
+            tau_sq: bool = False, T_norm: int | None = None):
     """Full forward: returns (loss, lse [T], kl [T]); loss carries the tau^2
     factor when ``tau_sq``, kl does not.
+
+    ``T_norm`` (default T) is the number of positions the mean divides by:
+    when these T rows are one shard of a batch of T_norm positions, the loss
+    returned is this shard's part of the batch's mean, (1/T_norm) sum_t KL_t.
 
     ``row_block`` only bounds host memory (each row is independent); results do
     not depend on it except through fp64 rounding of the final mean.
@@ -192,7 +196,8 @@ def forward(h, W, vals, idx, tau: float = 1.0, row_block: int = 256, cache: str 
         _, a, l = _row_block_stats(h64[t0:t1], W64, tau)
         lse[t0:t1] = l
         kl[t0:t1] = _kl_from(a, l, p[t0:t1], idx[t0:t1])
-    return loss_weight(tau, tau_sq) * (kl.sum() / T), lse, kl
+    n = T if T_norm is None else T_norm
+    return loss_weight(tau, tau_sq) * (kl.sum() / n), lse, kl
 
 
 def forward_rows(h, W, vals, idx, tau: float, rows, cache: str = "logits"):
@@ -217,13 +222,15 @@ def _dz_block(a, lse, p, S, idx, scale):
 
 
 def backward(h, W, vals, idx, tau: float = 1.0, g: float = 1.0, row_block: int = 256,
-             cache: str = "logits", tau_sq: bool = False):
-    """Full backward: returns (dH [T,d], dW [V,d]) in fp64."""
+             cache: str = "logits", tau_sq: bool = False, T_norm: int | None = None):
+    """Full backward: returns (dH [T,d], dW [V,d]) in fp64.  ``T_norm`` as in
+    ``forward``: the gradients of this shard's part of a batch's mean."""
     h64, W64 = _as_f64(h), _as_f64(W)
     idx = np.asarray(idx)
     T = h64.shape[0]
     p, S, _ = teacher_distribution(vals, tau, cache)
-    scale = loss_weight(tau, tau_sq) * g / (T * tau)
+    n = T if T_norm is None else T_norm
+    scale = loss_weight(tau, tau_sq) * g / (n * tau)
     dH = np.empty_like(h64)
     dW = np.zeros_like(W64)
     for t0 in range(0, T, row_block):

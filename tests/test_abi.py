@@ -244,3 +244,35 @@ def test_workspace_size_reports_zero_when_it_cannot_be_represented(lib):
                 ws_bytes=(1 << 64) - 1) == kd.KD_ERR_WORKSPACE
     assert _bwd(T=1 << 30, d=d, V=4096, K=1, chunk=1 << 30, dtype=kd.KD_DTYPE_F32,
                 ws_bytes=(1 << 64) - 1) == kd.KD_ERR_WORKSPACE
+
+
+def _fwd_shard(**kw):
+    a = dict(h=FAKE, W=FAKE, dtype=kd.KD_DTYPE_BF16, T=256, d=256, V=4096, vals=FAKE, idx=FAKE,
+             K=16, chunk=64, tau=1.0, flags=0, T_total=512, loss=FAKE, lse=FAKE, kl=None, ws=FAKE,
+             ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return kd.kd_fused_kl_fwd_shard(a["h"], a["W"], a["dtype"], a["T"], a["d"], a["V"], a["vals"],
+                                    a["idx"], a["K"], a["chunk"], a["tau"], a["flags"], a["T_total"],
+                                    a["loss"], a["lse"], a["kl"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+def _bwd_shard(**kw):
+    a = dict(h=FAKE, W=FAKE, dtype=kd.KD_DTYPE_BF16, T=256, d=256, V=4096, vals=FAKE, idx=FAKE,
+             K=16, chunk=64, tau=1.0, flags=0, T_total=512, lse=FAKE, g=None, dH=FAKE, dW=FAKE,
+             acc=0, ws=FAKE, ws_bytes=1 << 40, stream=None)
+    a.update(kw)
+    return kd.kd_fused_kl_bwd_shard(a["h"], a["W"], a["dtype"], a["T"], a["d"], a["V"], a["vals"],
+                                    a["idx"], a["K"], a["chunk"], a["tau"], a["flags"], a["T_total"],
+                                    a["lse"], a["g"], a["dH"], a["dW"], a["acc"], a["ws"],
+                                    a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("call", [_fwd_shard, _bwd_shard])
+def test_shard_validation(lib, call):
+    assert call(T_total=255) == kd.KD_ERR_INVALID_ARG        # fewer batch positions than rows
+    assert call(T_total=0) == kd.KD_ERR_INVALID_ARG
+    assert call(T_total=1 << 40) == kd.KD_ERR_UNSUPPORTED
+    assert call(flags=0x80) == kd.KD_ERR_INVALID_ARG
+    assert call(h=None) == kd.KD_ERR_INVALID_ARG             # the shared input checks
+    assert call(K=1025) == kd.KD_ERR_UNSUPPORTED
+    assert call(ws_bytes=16) == kd.KD_ERR_WORKSPACE
