@@ -203,10 +203,23 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // The next kernel in the stream may start launching now: its CTAs take an SM
+  // only as this grid's CTAs leave (shared memory), or sit beside them and
+  // wait for this grid to complete before touching what it writes.
+  griddep_launch_dependents();
+  // What this grid reads or overwrites that earlier kernels of the stream
+  // produced or still read: the epilogue's inputs (the sorted cache, lse) and
+  // every output region; for dH and dW also the A operand (dz).  The operands
+  // h and W of the projections are the caller's inputs, final before the
+  // call's first kernel (launched in plain stream order) started, so their
+  // loads need not wait: the mainloop of the first tiles overlaps the tail of
+  // the kernel before.
+  constexpr bool kOperandsWait = (EPI == EPI_STORE_PARTIAL || EPI == EPI_ACCUM_W);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
+      if (kOperandsWait) griddep_wait();
       int stage = 0;
       uint32_t phase = 0, armed = 0, last_par = 0;
       bool ok = true;
@@ -315,6 +328,7 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
+    griddep_wait();
     const int quad = warp & 3;
     unsigned char* boxes = sEpi + (warp - 2) * 2 * EPI_BUF_BYTES;
     const uint32_t tempty_leader0 = mapa_shared(smem_u32(&tempty[0]), 0);

@@ -132,6 +132,8 @@ __global__ void __launch_bounds__(256)
 combine_kernel(const float4* __restrict__ partials, int rows, int n_tiles, int64_t row0,
                float zscale, float inv_tau, const float2* __restrict__ stats,
                float* __restrict__ lse, float* __restrict__ kl) {
+  griddep_launch_dependents();
+  griddep_wait();                       // the chunk's GEMM has written the partials
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= rows) return;
@@ -170,32 +172,38 @@ combine_kernel(const float4* __restrict__ partials, int rows, int n_tiles, int64
 }
 
 // dH rows of a chunk = sum over K-splits of the fp32 partials, in split order.
-// One thread per 4 consecutive elements (d % 8 == 0).
+// One thread per 4 consecutive elements (d % 8 == 0), grid-stride over a grid
+// small enough to be resident at once (so that the next kernel can launch
+// while this one waits for the dH GEMM).
 template <typename Elem>
 __global__ void __launch_bounds__(256)
 dh_reduce_kernel(const float* __restrict__ part, int k_split, int64_t split_rows, int rows,
                  int64_t d, Elem* __restrict__ dH) {
-  const int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  griddep_launch_dependents();
+  griddep_wait();                       // the dH GEMM has written the partials
   const int64_t per_row = d / 4;
-  if (q >= static_cast<int64_t>(rows) * per_row) return;
-  const int64_t m = q / per_row, j = (q - m * per_row) * 4;
-  float4 acc = reinterpret_cast<const float4*>(part + m * d + j)[0];
-  for (int s = 1; s < k_split; ++s) {
-    const float4 x = reinterpret_cast<const float4*>(part + (s * split_rows + m) * d + j)[0];
-    acc.x += x.x;
-    acc.y += x.y;
-    acc.z += x.z;
-    acc.w += x.w;
-  }
-  if constexpr (sizeof(Elem) == 4) {
-    reinterpret_cast<float4*>(dH + m * d + j)[0] = acc;
-  } else {
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
-    uint2 w;
-    w.x = *reinterpret_cast<uint32_t*>(&lo);
-    w.y = *reinterpret_cast<uint32_t*>(&hi);
-    reinterpret_cast<uint2*>(dH + m * d + j)[0] = w;
+  const int64_t n = static_cast<int64_t>(rows) * per_row;
+  for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < n;
+       q += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = q / per_row, j = (q - m * per_row) * 4;
+    float4 acc = reinterpret_cast<const float4*>(part + m * d + j)[0];
+    for (int s = 1; s < k_split; ++s) {
+      const float4 x = reinterpret_cast<const float4*>(part + (s * split_rows + m) * d + j)[0];
+      acc.x += x.x;
+      acc.y += x.y;
+      acc.z += x.z;
+      acc.w += x.w;
+    }
+    if constexpr (sizeof(Elem) == 4) {
+      reinterpret_cast<float4*>(dH + m * d + j)[0] = acc;
+    } else {
+      __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y);
+      __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z, acc.w);
+      uint2 w;
+      w.x = *reinterpret_cast<uint32_t*>(&lo);
+      w.y = *reinterpret_cast<uint32_t*>(&hi);
+      reinterpret_cast<uint2*>(dH + m * d + j)[0] = w;
+    }
   }
 }
 
@@ -283,6 +291,27 @@ bool make_out_map(CUtensorMap* map, const void* base, bool f32, uint64_t inner, 
                   f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
+// Launches a small kernel with programmatic stream serialization (it may start
+// while the kernel before it runs, and waits inside for that kernel's results).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, args...);
+  count_launch();
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 // Clusters of two CTAs that can be resident at once for this kernel, cached
 // per device (atomics: calls may come from several host threads).
 constexpr int KD_MAX_DEVICES = 64;
@@ -333,13 +362,17 @@ cudaError_t launch_gemm2(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
   cfg.blockDim = dim3(GEMM_THREADS);
   cfg.dynamicSmemBytes = GEMM2_SMEM_BYTES;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // may start while the kernel before it runs (the kernel waits inside for
+  // whatever that kernel writes)
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   profile_before(kKind[EPI], 2.0 * g.M * static_cast<double>(g.N) * g.K, s);
   e = cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, g);
   count_launch();
@@ -490,10 +523,10 @@ static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t T_nor
         cudaSuccess)
       return KD_ERR_CUDA;
     const int cblocks = cdiv(rows * 32, 256);
-    combine_kernel<<<cblocks, 256, 0, s>>>(part, static_cast<int>(rows), g.n_tiles, c0, zscale,
-                                           inv_tau, stats, lse, kl);
-    count_launch();
-    if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+    if (launch_pdl(combine_kernel, static_cast<unsigned>(cblocks), 256u, s,
+                   static_cast<const float4*>(part), static_cast<int>(rows), g.n_tiles, c0, zscale,
+                   inv_tau, static_cast<const float2*>(stats), lse, kl) != cudaSuccess)
+      return KD_ERR_CUDA;
   }
   mean_kernel<<<1, 1024, 0, s>>>(kl, T, T_norm, loss_weight(tau, flags), loss);
   count_launch();
@@ -607,11 +640,13 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t T_nor
         return KD_ERR_CUDA;
       {
         const int64_t n4 = rows * (d / 4);
-        dh_reduce_kernel<Elem><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, s>>>(
-            hpart, gh.k_split, L.rows_pad, static_cast<int>(rows), d,
-            static_cast<Elem*>(dH) + c0 * d);
-        count_launch();
-        if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
+        int64_t blocks = (n4 + 255) / 256;
+        if (blocks > 2 * static_cast<int64_t>(num_sms)) blocks = 2 * static_cast<int64_t>(num_sms);
+        if (launch_pdl(dh_reduce_kernel<Elem>, static_cast<unsigned>(blocks), 256u, s,
+                       static_cast<const float*>(hpart), gh.k_split,
+                       static_cast<int64_t>(L.rows_pad), static_cast<int>(rows), d,
+                       static_cast<Elem*>(dH) + c0 * d) != cudaSuccess)
+          return KD_ERR_CUDA;
       }
     }
 

@@ -246,10 +246,9 @@ __device__ __forceinline__ void for_each_elem(const uint16_t* __restrict__ row, 
 }
 
 // Appends one element to the survivor buffer if it passes the threshold (the
-// exact per-element test; rarely reached from the streaming pass).
-__device__ __forceinline__ void offer(TopkSmem& sm, uint32_t bits, uint32_t i, float tf,
-                                     bool take_all) {
-  if (take_all || bf16_bits_to_float(bits) >= tf) {
+// exact per-element test, for the row's unaligned head and ragged tail).
+__device__ __forceinline__ void offer(TopkSmem& sm, uint32_t bits, uint32_t i, float tf) {
+  if (bf16_bits_to_float(bits) >= tf) {
     const uint32_t pos = atomicAdd(&sm.n_cand, 1u);
     if (pos < TK_CAND_CAP) sm.cand[pos] = composite(bf16_order_key(bits), i, bits);
   }
@@ -257,8 +256,7 @@ __device__ __forceinline__ void offer(TopkSmem& sm, uint32_t bits, uint32_t i, f
 
 // Exact test of the 8 elements of a screened vector: a pass mask built without
 // branches, then one append per passing element (usually one).
-__device__ __forceinline__ void offer8(TopkSmem& sm, uint4 q, uint32_t base, float tf,
-                                       bool take_all) {
+__device__ __forceinline__ void offer8(TopkSmem& sm, uint4 q, uint32_t base, float tf) {
   const uint32_t w[4] = {q.x, q.y, q.z, q.w};
   uint32_t m = 0;
 #pragma unroll
@@ -266,7 +264,6 @@ __device__ __forceinline__ void offer8(TopkSmem& sm, uint4 q, uint32_t base, flo
     m |= (__uint_as_float(w[e] << 16) >= tf ? 1u : 0u) << (2 * e);
     m |= (__uint_as_float(w[e] & 0xFFFF0000u) >= tf ? 1u : 0u) << (2 * e + 1);
   }
-  if (take_all) m = 0xFFu;
   while (m) {
     const int b = __ffs(m) - 1;
     m &= m - 1;
@@ -287,106 +284,179 @@ __device__ __forceinline__ __nv_bfloat162 max8_packed(uint4 q) {
   return __hmax2(__hmax2(as_bf162(q.x), as_bf162(q.y)), __hmax2(as_bf162(q.z), as_bf162(q.w)));
 }
 
-// True if some element of the pair is >= tb (a NaN compares false).
-__device__ __forceinline__ bool any_ge(__nv_bfloat162 m, __nv_bfloat16 tb) {
-  return __hge(__hmax(__low2bfloat16(m), __high2bfloat16(m)), tb);
+// False only if both halves of m are below tb (one paired compare); a NaN
+// half passes the screen and is rejected by the exact per-element test.
+__device__ __forceinline__ uint32_t screen_bit(__nv_bfloat162 m, uint32_t tb2) {
+  uint32_t r;
+  asm("{\n\t.reg .pred p, q;\n\t"
+      "setp.lt.bf16x2 p|q, %1, %2;\n\t"
+      "and.pred p, p, q;\n\t"
+      "selp.u32 %0, 0, 1, p;\n\t}"
+      : "=r"(r)
+      : "r"(*reinterpret_cast<uint32_t*>(&m)), "r"(tb2));
+  return r;
 }
 
-// The streaming pass: every element of the row meets the threshold once.
-// Each thread holds TK_UNROLL 16-byte vectors (64 elements) in flight, and each
-// vector is screened by its packed maximum (three max.bf16x2 and one bf16
-// compare; NaN operands are ignored by max.bf16x2, and tf is a bf16 value, or
-// -inf or 0, so the bf16 compare is exact).  A vector that may hold a survivor
-// is not tested on the spot, which would make the whole warp run the exact
-// test for one lane: its lane appends it to the warp's staging buffer
-// (position from a ballot), and once the buffer is full, and at the end, the
-// warp runs the exact test on up to 32 staged vectors at once, one per lane.
-// The row is walked in warp-uniform steps so that every lane takes part in
-// every ballot.
-__device__ __forceinline__ void stream_survivors(TopkSmem& sm, const uint16_t* __restrict__ row,
-                                                 int64_t V, float tf, bool take_all,
-                                                 uint32_t* status) {
-  const uintptr_t addr = reinterpret_cast<uintptr_t>(row);
-  int64_t head = ((16 - (addr & 15)) & 15) >> 1;
-  if (head > V) head = V;
-  for (int64_t i = threadIdx.x; i < head; i += TK_THREADS)
-    offer(sm, row[i], static_cast<uint32_t>(i), tf, take_all);
-  const int64_t nvec = (V - head) >> 3;
-  const uint4* vp = reinterpret_cast<const uint4*>(row + head);
-  const __nv_bfloat16 tb = __float2bfloat16_rn(tf);
-  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const uint32_t lanes_below = (1u << lane) - 1u;
-  uint4* sq = sm.stage_q[wid];
-  uint32_t* sb = sm.stage_base[wid];
-  int cnt = 0;                                      // staged vectors (warp-uniform)
-  for (int64_t jb = 0; jb < nvec; jb += static_cast<int64_t>(TK_THREADS) * TK_UNROLL) {
-    const int64_t j0 = jb + threadIdx.x;
-    const bool full = jb + static_cast<int64_t>(TK_THREADS) * TK_UNROLL <= nvec;  // warp-uniform
-    uint4 q[TK_UNROLL];
-    if (full) {
+// L2 prefetch of `bytes` (a multiple of 16) from a 16-byte-aligned global
+// address, issued by one thread as a single bulk operation.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
+// Stage this lane's screened vectors (bit u of m: vector q[u] may hold a
+// survivor; its first element is at row index base + u*TK_THREADS*8) into the
+// warp's 32-entry buffer at positions from a warp prefix sum; when the buffer
+// would overflow, the warp first runs the exact test on what it holds.  A
+// batch of more than 32 vectors (only rows with very many survivors close
+// together) is staged vector slot by vector slot instead, at most 32 at a
+// time.  Warp-uniform.
+__device__ __forceinline__ void flush_stage(TopkSmem& sm, const uint4* sq, const uint32_t* sb,
+                                            uint32_t& cnt, float tf, int lane) {
+  __syncwarp();
+  if (static_cast<uint32_t>(lane) < cnt) offer8(sm, sq[lane], sb[lane], tf);
+  __syncwarp();
+  cnt = 0;
+}
+
+__device__ __forceinline__ void stage_vectors(TopkSmem& sm, uint4* sq, uint32_t* sb, uint32_t& cnt,
+                                              uint32_t m, const uint4 (&q)[TK_UNROLL],
+                                              uint32_t base, float tf, int lane, uint32_t* status) {
+  const uint32_t c = __popc(m);
+  uint32_t x = c;
 #pragma unroll
-      for (int u = 0; u < TK_UNROLL; ++u) q[u] = __ldcs(vp + j0 + u * TK_THREADS);
-    } else {
-#pragma unroll
-      for (int u = 0; u < TK_UNROLL; ++u) {
-        const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
-        q[u] = j < nvec ? __ldcs(vp + j) : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u,
-                                                     0xFF80FF80u);   // -inf
-      }
-    }
-    // The next step's vectors into L2 while this step's are screened (a hint:
-    // no registers held, nothing waits on it).
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  const uint32_t total = __shfl_sync(0xffffffffu, x, 31);
+  if (total > 32u) {
+    const uint32_t lanes_below = (1u << lane) - 1u;
 #pragma unroll
     for (int u = 0; u < TK_UNROLL; ++u) {
-      const int64_t j = j0 + static_cast<int64_t>(TK_THREADS) * TK_UNROLL +
-                        static_cast<int64_t>(u) * TK_THREADS;
-      if (j < nvec) asm volatile("prefetch.global.L2 [%0];" ::"l"(vp + j));
-    }
-#pragma unroll
-    for (int u = 0; u < TK_UNROLL; ++u) {
-      const int64_t j = j0 + static_cast<int64_t>(u) * TK_THREADS;
-      const bool pass = (full || j < nvec) && (take_all || any_ge(max8_packed(q[u]), tb));
+      const bool pass = (m >> u) & 1u;
       const uint32_t b = __ballot_sync(0xffffffffu, pass);
       if (b) {
-        const int nb = __popc(b);
-        if (cnt + nb > 32) {                        // buffer full: test what it holds
-          __syncwarp();
-          if (lane < cnt) offer8(sm, sq[lane], sb[lane], tf, take_all);
-          __syncwarp();
-          cnt = 0;
-        }
+        const uint32_t nb = __popc(b);
+        if (cnt + nb > 32u) flush_stage(sm, sq, sb, cnt, tf, lane);
         if (pass) {
-          const int pos = cnt + __popc(b & lanes_below);
-          KD_CHECK(pos < 32, status);
+          const uint32_t pos = cnt + __popc(b & lanes_below);
           sq[pos] = q[u];
-          sb[pos] = static_cast<uint32_t>(head + (j << 3));
+          sb[pos] = base + u * TK_THREADS * 8;
         }
         cnt += nb;
       }
     }
+    return;
   }
-  __syncwarp();
-  if (lane < cnt) offer8(sm, sq[lane], sb[lane], tf, take_all);
-  __syncwarp();
-  for (int64_t i = head + (nvec << 3) + threadIdx.x; i < V; i += TK_THREADS)
-    offer(sm, row[i], static_cast<uint32_t>(i), tf, take_all);
+  if (cnt + total > 32u) flush_stage(sm, sq, sb, cnt, tf, lane);
+  uint32_t pos = cnt + x - c;
+#pragma unroll
+  for (int u = 0; u < TK_UNROLL; ++u) {
+    if ((m >> u) & 1u) {
+      KD_CHECK(pos < 32u, status);
+      sq[pos] = q[u];
+      sb[pos] = base + u * TK_THREADS * 8;
+      ++pos;
+    }
+  }
+  cnt += total;
+}
+
+// The streaming pass: every element of the row meets the threshold once.
+// Each thread holds TK_UNROLL 16-byte vectors (64 elements) in flight, and each
+// vector is screened by its packed maximum: three max.bf16x2 and one paired
+// bf16x2 compare against tf (NaN operands are ignored by max.bf16x2, and tf
+// is a bf16 value, never -inf or NaN, so the screen passes every vector that
+// holds a survivor).  The screens of a thread's vectors form a bit mask; a
+// vector that may hold a survivor is not tested on the spot, which would make
+// the whole warp run the exact test for one lane: it goes to the warp's
+// staging buffer, and once the buffer is full, and at the end, the warp runs
+// the exact test on up to 32 staged vectors at once, one per lane.
+// One thread keeps the CTA's stream two steps (64 KB) ahead in L2 with single
+// bulk prefetches; near the end of the row they run on into the first steps of
+// the CTA's next row (`next_vp`, or null; given only when every row starts on
+// 16 bytes, so the next row has the same full steps), so that HBM keeps working
+// for this CTA while it selects and samples.  Every prefetch lies inside a full
+// step of this row or of the next.  Indices are 32-bit (V < 2^31).
+__device__ __forceinline__ void stream_survivors(TopkSmem& sm, const uint16_t* __restrict__ row,
+                                                 uint32_t V, float tf, const uint4* next_vp,
+                                                 uint32_t* status) {
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const uintptr_t addr = reinterpret_cast<uintptr_t>(row);
+  uint32_t head = static_cast<uint32_t>(((16 - (addr & 15)) & 15) >> 1);
+  if (head > V) head = V;
+  for (uint32_t i = tid; i < head; i += TK_THREADS) offer(sm, row[i], i, tf);
+  const uint32_t nvec = (V - head) >> 3;
+  const uint4* vp = reinterpret_cast<const uint4*>(row + head);
+  const __nv_bfloat16 tb = __float2bfloat16_rn(tf);
+  const uint32_t tb2 = static_cast<uint32_t>(__bfloat16_as_ushort(tb)) * 0x10001u;
+  uint4* sq = sm.stage_q[wid];
+  uint32_t* sb = sm.stage_base[wid];
+  uint32_t cnt = 0;                                  // staged vectors (warp-uniform)
+  constexpr uint32_t STEP = TK_THREADS * TK_UNROLL;  // vectors per CTA step
+  const uint32_t nfull = nvec / STEP;
+  if (tid == 0 && nfull > 1) bulk_prefetch_l2(vp + STEP, STEP * 16);
+  for (uint32_t it = 0; it < nfull; ++it) {
+    const uint4* p = vp + it * STEP + tid;
+    uint4 q[TK_UNROLL];
+#pragma unroll
+    for (int u = 0; u < TK_UNROLL; ++u) q[u] = __ldcs(p + u * TK_THREADS);
+    uint32_t m = 0;
+#pragma unroll
+    for (int u = 0; u < TK_UNROLL; ++u) m |= screen_bit(max8_packed(q[u]), tb2) << u;
+    if (__any_sync(0xffffffffu, m != 0u))
+      stage_vectors(sm, sq, sb, cnt, m, q, head + (it * STEP + tid) * 8, tf, lane, status);
+    if (tid == 0) {          // the step after next, in this row or the next one
+      const uint32_t s2 = it + 2;
+      if (s2 < nfull)
+        bulk_prefetch_l2(p + 2 * STEP, STEP * 16);   // thread 0's p is vp + it*STEP
+      else if (next_vp && s2 - nfull < nfull)     // the next row has the same nfull
+        bulk_prefetch_l2(next_vp + (s2 - nfull) * STEP, STEP * 16);
+    }
+  }
+  if (nfull * STEP < nvec) {  // the last, partial step: absent vectors read as -inf
+    const uint32_t j0 = nfull * STEP + tid;
+    uint4 q[TK_UNROLL];
+#pragma unroll
+    for (int u = 0; u < TK_UNROLL; ++u) {
+      const uint32_t j = j0 + u * TK_THREADS;
+      q[u] = j < nvec ? __ldcs(vp + j)
+                      : make_uint4(0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u, 0xFF80FF80u);
+    }
+    uint32_t m = 0;
+#pragma unroll
+    for (int u = 0; u < TK_UNROLL; ++u) m |= screen_bit(max8_packed(q[u]), tb2) << u;
+    if (__any_sync(0xffffffffu, m != 0u))
+      stage_vectors(sm, sq, sb, cnt, m, q, head + j0 * 8, tf, lane, status);
+  }
+  flush_stage(sm, sq, sb, cnt, tf, lane);
+  for (uint32_t i = head + (nvec << 3) + tid; i < V; i += TK_THREADS) offer(sm, row[i], i, tf);
 }
 
 __global__ void __launch_bounds__(TK_THREADS, 4)
 topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int K,
-                 float* __restrict__ out_vals, int32_t* __restrict__ out_idx,
-                 uint32_t* __restrict__ status) {
+                 uint32_t sample_target, int fast_sample, float* __restrict__ out_vals,
+                 int32_t* __restrict__ out_idx, uint32_t* __restrict__ status) {
   extern __shared__ __align__(16) unsigned char tk_smem_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_smem_raw);
   const int tid = threadIdx.x;
+  const bool rows_aligned = (V & 7) == 0;            // every row starts on 16 bytes
 
   for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
     const uint16_t* row = logits + t * V;
 
     // ---- 1. sample threshold -------------------------------------------------
-    // L = the key of the target-th largest sample element, found in two levels
-    // of 256 bins: the key's high byte, then its low byte inside the chosen
-    // high-byte bin (bin 0 holds the highest keys).
+    // L = the key of the target-th largest sample key, found in two levels of
+    // 256 bins: the key's high byte, then its low byte inside the chosen
+    // high-byte bin (bin 0 holds the highest keys).  The sample is the row's
+    // first TK_SAMPLE elements (all of it when V <= TK_SAMPLE, with target K).
+    // On the fast path (long aligned rows, small targets) each thread
+    // contributes one key, the largest of its 16 sample elements (a packed
+    // bf16 maximum, NaN ignored), and the target-th largest of those 256 keys
+    // is L: at most the target-th largest sample element, so the expected
+    // number of survivors is about the same (about 3K) and never smaller.  Any
+    // L gives the exact result: survivors are every element with key >= L,
+    // and rows with fewer than K of them take the fallback.
     sm.hist[tid] = 0u;
     sm.hist[TK_THREADS + tid] = 0u;
     if (tid == 0) {
@@ -394,74 +464,74 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
       sm.n_sel = 0;
     }
     __syncthreads();
-    const int64_t S = V < TK_SAMPLE ? V : TK_SAMPLE;
-    // The sample's keys stay in registers: SAMPLE_PER_THREAD per thread, loaded
-    // in one batch (16-byte vectors when the row is aligned and long enough).
-    uint32_t skey[SAMPLE_PER_THREAD];
-    if (S == TK_SAMPLE && (reinterpret_cast<uintptr_t>(row) & 15u) == 0) {
+    const uint32_t target = sample_target;
+    uint32_t L;
+    if (fast_sample) {
       const uint4* vp = reinterpret_cast<const uint4*>(row);
-      uint4 q[SAMPLE_PER_THREAD / 8];
+      const uint4 q0 = vp[tid], q1 = vp[tid + TK_THREADS];
+      __nv_bfloat162 mm = __hmax2(max8_packed(q0), max8_packed(q1));
+      const uint32_t w = *reinterpret_cast<uint32_t*>(&mm);
+      const uint32_t k0 = bf16_order_key(w & 0xFFFFu), k1 = bf16_order_key(w >> 16);
+      const uint32_t key = k0 > k1 ? k0 : k1;
+      atomicAdd(&sm.hist[255u - (key >> 8)], 1u);
+      __syncthreads();
+      find_bin_256(sm.hist, target, &sm.thr_bin, &sm.thr_above, &sm.n_sel);
+      __syncthreads();
+      KD_CHECK(sm.thr_bin < 256u, status);
+      const uint32_t hb = 255u - sm.thr_bin;          // high byte of L
+      const uint32_t above_hb = sm.thr_above;
+      if ((key >> 8) == hb) atomicAdd(&sm.hist[TK_THREADS + 255u - (key & 255u)], 1u);
+      __syncthreads();
+      find_bin_256(sm.hist + TK_THREADS, target - above_hb, &sm.thr_bin, &sm.thr_above,
+                   &sm.n_sel);
+      __syncthreads();
+      KD_CHECK(sm.thr_bin < 256u, status);
+      L = (hb << 8) | (255u - sm.thr_bin);
+    } else {
+      const int64_t S = V < TK_SAMPLE ? V : TK_SAMPLE;
+      // The sample's keys stay in registers: SAMPLE_PER_THREAD per thread.
+      uint32_t skey[SAMPLE_PER_THREAD];
+      {
+        uint32_t raw[SAMPLE_PER_THREAD];
 #pragma unroll
-      for (int u = 0; u < SAMPLE_PER_THREAD / 8; ++u) q[u] = vp[tid + u * TK_THREADS];
+        for (int u = 0; u < SAMPLE_PER_THREAD; ++u) {
+          const int64_t i = tid + static_cast<int64_t>(u) * TK_THREADS;
+          raw[u] = i < S ? row[i] : 0u;
+        }
 #pragma unroll
-      for (int u = 0; u < SAMPLE_PER_THREAD / 8; ++u) {
-        const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          skey[u * 8 + 2 * e] = bf16_order_key(w[e] & 0xFFFFu);
-          skey[u * 8 + 2 * e + 1] = bf16_order_key(w[e] >> 16);
+        for (int u = 0; u < SAMPLE_PER_THREAD; ++u) {
+          const int64_t i = tid + static_cast<int64_t>(u) * TK_THREADS;
+          skey[u] = i < S ? bf16_order_key(raw[u]) : 0xFFFFFFFFu;   // marker: not sampled
         }
       }
-    } else {
-      uint32_t raw[SAMPLE_PER_THREAD];
 #pragma unroll
-      for (int u = 0; u < SAMPLE_PER_THREAD; ++u) {
-        const int64_t i = tid + static_cast<int64_t>(u) * TK_THREADS;
-        raw[u] = i < S ? row[i] : 0u;
-      }
+      for (int u = 0; u < SAMPLE_PER_THREAD; ++u)
+        if (skey[u] != 0xFFFFFFFFu) atomicAdd(&sm.hist[255u - (skey[u] >> 8)], 1u);
+      __syncthreads();
+      // (target <= S: either S == V >= K and target == K, or V > 4096 >= 3K)
+      find_bin_256(sm.hist, target, &sm.thr_bin, &sm.thr_above, &sm.n_sel);
+      __syncthreads();
+      KD_CHECK(sm.thr_bin < 256u, status);
+      const uint32_t hb = 255u - sm.thr_bin;          // high byte of L
+      const uint32_t above_hb = sm.thr_above;
 #pragma unroll
-      for (int u = 0; u < SAMPLE_PER_THREAD; ++u) {
-        const int64_t i = tid + static_cast<int64_t>(u) * TK_THREADS;
-        skey[u] = i < S ? bf16_order_key(raw[u]) : 0xFFFFFFFFu;   // marker: not sampled
-      }
+      for (int u = 0; u < SAMPLE_PER_THREAD; ++u)
+        if (skey[u] != 0xFFFFFFFFu && (skey[u] >> 8) == hb)
+          atomicAdd(&sm.hist[TK_THREADS + 255u - (skey[u] & 255u)], 1u);
+      __syncthreads();
+      find_bin_256(sm.hist + TK_THREADS, target - above_hb, &sm.thr_bin, &sm.thr_above,
+                   &sm.n_sel);
+      __syncthreads();
+      KD_CHECK(sm.thr_bin < 256u, status);
+      L = (hb << 8) | (255u - sm.thr_bin);            // candidate iff order key >= L
     }
-#pragma unroll
-    for (int u = 0; u < SAMPLE_PER_THREAD; ++u)
-      if (skey[u] != 0xFFFFFFFFu) atomicAdd(&sm.hist[255u - (skey[u] >> 8)], 1u);
-    __syncthreads();
-    uint32_t target;
-    if (S == V) {
-      target = static_cast<uint32_t>(K);
-    } else {
-      // about 3K expected survivors over the whole row
-      const double want = 3.0 * K * static_cast<double>(S) / static_cast<double>(V);
-      target = static_cast<uint32_t>(ceil(want));
-      if (target < 1u) target = 1u;
-    }
-    // (target <= S: either S == V >= K, or V > 4096 >= 3K)
-    find_bin_256(sm.hist, target, &sm.thr_bin, &sm.thr_above, &sm.n_sel);
-    __syncthreads();
-    KD_CHECK(sm.thr_bin < 256u, status);
-    const uint32_t hb = 255u - sm.thr_bin;            // high byte of L
-    const uint32_t above_hb = sm.thr_above;
-#pragma unroll
-    for (int u = 0; u < SAMPLE_PER_THREAD; ++u)
-      if (skey[u] != 0xFFFFFFFFu && (skey[u] >> 8) == hb)
-        atomicAdd(&sm.hist[TK_THREADS + 255u - (skey[u] & 255u)], 1u);
-    __syncthreads();
-    find_bin_256(sm.hist + TK_THREADS, target - above_hb, &sm.thr_bin, &sm.thr_above, &sm.n_sel);
-    __syncthreads();
-    KD_CHECK(sm.thr_bin < 256u, status);
-    const uint32_t L = (hb << 8) | (255u - sm.thr_bin);   // candidate iff order key >= L
     if (tid == 0) sm.n_sel = 0u;
     // Float threshold equivalent on non-NaN values: key >= L <=> x >= tf.
+    // A threshold at or below -inf (the sample's top is NaN or -inf) would
+    // keep almost the whole row: such rows go straight to the exact fallback.
+    const bool screen = L > 0x7Fu;
     float tf = 0.f;
-    bool take_all = false;
-    if (L == 0u) {
-      take_all = true;                              // threshold inside the NaN bin
-    } else if (L <= 0x7Fu) {
-      tf = -INFINITY;                               // every non-NaN value qualifies
-    } else if (L == 0x7FFFu) {
+    if (L == 0x7FFFu) {
       tf = 0.f;                                     // between -0's raw key and +0
     } else if (L < 0x8000u) {
       tf = bf16_bits_to_float((~L) & 0xFFFFu);      // the negative value with key L
@@ -470,42 +540,103 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
     }
 
     // ---- 2. stream the row, keep survivors ------------------------------------
-    stream_survivors(sm, row, V, tf, take_all, status);
+    if (screen) {
+      const uint4* next_vp = (rows_aligned && t + gridDim.x < T)
+                                 ? reinterpret_cast<const uint4*>(logits + (t + gridDim.x) * V)
+                                 : nullptr;
+      stream_survivors(sm, row, static_cast<uint32_t>(V), tf, next_vp, status);
+    }
     __syncthreads();
-    const uint32_t n = sm.n_cand;
+    const uint32_t n = screen ? sm.n_cand : 0u;
 
     if (n >= static_cast<uint32_t>(K) && n <= static_cast<uint32_t>(TK_CAND_CAP)) {
       // ---- 3. exact select among survivors -------------------------------------
-      // (a) the exact K-th largest key among the survivors.  Every survivor's
-      //     key is >= L.  When they span fewer than TK_THREADS keys (the usual
-      //     case: few bf16 values lie near the top of a row) one histogram of
-      //     key - L, one bin per thread, and one block scan give it; otherwise
-      //     a 4096-bin histogram of key >> 4, then the 16 keys of the
-      //     threshold bin.
-      static_assert(TK_THREADS <= TK_BINS, "narrow histogram lives in hist");
+      // Every survivor's key is >= L.  When they span fewer than 256 keys (the
+      // usual case: few bf16 values lie near the top of a row), one histogram
+      // of key - L, bin 0 holding the highest key, orders them: its prefix sums
+      // are the first output slot of each key, the survivors are scattered into
+      // their key's bucket, and each one's output position is its bucket's first
+      // slot plus the number of bucket entries with a lower index.  Otherwise a
+      // 4096-bin histogram of key >> 4, then the 16 keys of the threshold bin,
+      // give the exact K-th key, and the survivors at or above it are ranked by
+      // counting.
+      static_assert(TK_THREADS == 256, "one narrow-histogram bin per thread");
+      uint32_t* nh = sm.hist;                        // [256] counts per key - L
+      uint32_t* nstart = sm.hist + 256;              // [256] first output slot per bin
+      uint32_t* nfill = sm.hist + 512;               // [256] entries placed per bin
       if (tid == 0) {
         sm.wide = 0u;
         sm.n_sel = 0u;
       }
-      sm.hist[tid] = 0u;
+      nh[tid] = 0u;
+      nfill[tid] = 0u;
       __syncthreads();
       for (int i = tid; i < static_cast<int>(n); i += TK_THREADS) {
         const uint32_t dk = comp_key(sm.cand[i]) - L;
-        if (dk < static_cast<uint32_t>(TK_THREADS))
-          atomicAdd(&sm.hist[TK_THREADS - 1 - dk], 1u);   // bin 0 = highest key
+        if (dk < 256u)
+          atomicAdd(&nh[255u - dk], 1u);
         else
           sm.wide = 1u;
       }
       __syncthreads();
       if (sm.wide == 0u) {
-        uint32_t* res = sm.warp_tot;                 // scratch: bin, above, through
-        find_bin_256(sm.hist, static_cast<uint32_t>(K), &res[0], &res[1], &res[2]);
-        __syncthreads();
-        KD_CHECK(res[0] < 256u, status);
-        if (tid == 0) {
-          sm.thr_bin = L + static_cast<uint32_t>(TK_THREADS - 1) - res[0];   // exact K-th key
-          sm.thr_above = res[2];                                            // survivors >= it
+        // warp 0: exclusive prefix of the 256 counts (8 bins per lane) and the
+        // bin where the count first reaches K (bins up to it: K plus ties)
+        if (tid < 32) {
+          const uint4 a4 = reinterpret_cast<const uint4*>(nh)[2 * tid];
+          const uint4 b4 = reinterpret_cast<const uint4*>(nh)[2 * tid + 1];
+          const uint32_t c[8] = {a4.x, a4.y, a4.z, a4.w, b4.x, b4.y, b4.z, b4.w};
+          uint32_t sum = 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) sum += c[j];
+          uint32_t incl = sum;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (tid >= o) incl += y;
+          }
+          uint32_t run = incl - sum;
+          if (KD_DEBUG && tid == 0) sm.thr_bin = 0xFFFFFFFFu;
+          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            nstart[8 * tid + j] = run;
+            if (run < static_cast<uint32_t>(K) && run + c[j] >= static_cast<uint32_t>(K)) {
+              sm.thr_bin = static_cast<uint32_t>(8 * tid + j);   // last bin kept
+              sm.thr_above = run + c[j];                          // entries kept (K + ties)
+            }
+            run += c[j];
+          }
         }
+        __syncthreads();
+        KD_CHECK(sm.thr_bin < 256u, status);
+        const uint32_t last_bin = sm.thr_bin;
+        const uint32_t ns = sm.thr_above;
+        if (ns <= static_cast<uint32_t>(TK_SEL_CAP)) {
+          for (int i = tid; i < static_cast<int>(n); i += TK_THREADS) {
+            const uint64_t c = sm.cand[i];
+            const uint32_t b = 255u - (comp_key(c) - L);
+            if (b <= last_bin) sm.sel[nstart[b] + atomicAdd(&nfill[b], 1u)] = c;
+          }
+          __syncthreads();
+          for (int s2 = tid; s2 < static_cast<int>(ns); s2 += TK_THREADS) {
+            const uint64_t c = sm.sel[s2];
+            const uint32_t b = 255u - (comp_key(c) - L);
+            const uint32_t lo = nstart[b], hi = lo + nh[b];
+            uint32_t r = lo;
+            for (uint32_t j = lo; j < hi; ++j) r += sm.sel[j] < c ? 1u : 0u;
+            if (r < static_cast<uint32_t>(K)) {
+              out_idx[t * K + r] = static_cast<int32_t>(comp_idx(c));
+              out_vals[t * K + r] = bf16_bits_to_float(comp_raw(c));
+            }
+          }
+          __syncthreads();
+          continue;
+        }
+        // more than TK_SEL_CAP entries tie at the K-th key: rank in place below
+        __syncthreads();                              // every thread has read thr_bin
+        if (tid == 0) sm.thr_bin = L + 255u - last_bin;   // exact K-th key
+        __syncthreads();
       } else {
         for (int b = tid; b < TK_BINS; b += TK_THREADS) sm.hist[b] = 0u;
         if (tid < 16) sm.hist16[tid] = 0u;
@@ -533,11 +664,11 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
           sm.thr_bin = (cb << 4) | nib;     // exact K-th key
           sm.thr_above = above + at;        // survivors with key >= it
         }
+        __syncthreads();
       }
-      __syncthreads();
       const uint32_t Tk = sm.thr_bin;
       const bool compact = sm.thr_above <= static_cast<uint32_t>(TK_SEL_CAP);
-      // (b) keep the survivors with key >= Tk (the top K plus ties at Tk);
+      // keep the survivors with key >= Tk (the top K plus ties at Tk);
       if (compact) {
         for (int i = tid; i < static_cast<int>(n); i += TK_THREADS) {
           const uint64_t c = sm.cand[i];
@@ -549,9 +680,9 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
         }
         __syncthreads();
       }
-      // (c) rank: the composites are distinct (they contain the index), so an
-      //     entry's output position is the number of entries ordered before
-      //     it; those below K write themselves there, already in order.
+      // rank: the composites are distinct (they contain the index), so an
+      // entry's output position is the number of entries ordered before it;
+      // those below K write themselves there, already in order.
       const uint64_t* set = compact ? sm.sel : sm.cand;
       const int ns = compact ? static_cast<int>(sm.n_sel) : static_cast<int>(n);
       KD_CHECK(ns >= K && (!compact || static_cast<uint32_t>(ns) == sm.thr_above), status);
@@ -689,8 +820,21 @@ cudaError_t launch_topk_bf16(const void* logits, int64_t T, int64_t V, int K, fl
   if (per_sm < 1) per_sm = 1;
   int64_t grid = static_cast<int64_t>(num_sms) * per_sm;
   if (grid > T) grid = T;
+  // Sample rank of the threshold: about 3K expected survivors over the row
+  // (all K when the sample is the whole row).  Integer ceil(3*K*S / V).
+  uint32_t target;
+  if (V <= TK_SAMPLE) {
+    target = static_cast<uint32_t>(K);
+  } else {
+    const int64_t num = 3 * static_cast<int64_t>(K) * TK_SAMPLE;
+    target = static_cast<uint32_t>((num + V - 1) / V);
+    if (target < 1u) target = 1u;
+  }
+  // one key per thread (the largest of its 16 sample elements) when rows are
+  // long and 16-byte aligned and the target is a small share of the 256 keys
+  const int fast = (V > TK_SAMPLE && (V & 7) == 0 && target <= 32u) ? 1 : 0;
   topk_bf16_kernel<<<static_cast<unsigned>(grid), TK_THREADS, smem, stream>>>(
-      static_cast<const uint16_t*>(logits), T, V, K, out_vals, out_idx, status);
+      static_cast<const uint16_t*>(logits), T, V, K, target, fast, out_vals, out_idx, status);
   count_launch();
   return cudaGetLastError();
 }
