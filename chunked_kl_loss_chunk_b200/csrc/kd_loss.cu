@@ -116,6 +116,142 @@ prep_kernel(const float* __restrict__ vals, const int32_t* __restrict__ idx, int
   }
 }
 
+// The same preparation for K <= 128, with the (index, p) pairs of a row held
+// in registers, four per lane (entry e = lane + 32*r), and sorted by a bitonic
+// network over the next power of two >= K whose exchanges are warp shuffles
+// (distances < 32) or register swaps (distances 32 and 64).  No shared memory,
+// so the kernel runs beside the first GEMM of the chunk loop, which may start
+// while it runs (programmatic dependent launch; it waits for this kernel's
+// results before reading them).
+constexpr int PREP_REG_MAXK = 128;
+
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t x, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(x), m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, static_cast<uint32_t>(x >> 32), m);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+__device__ __forceinline__ uint64_t shfl_u64(uint64_t x, int src) {
+  const uint32_t lo = __shfl_sync(0xffffffffu, static_cast<uint32_t>(x), src);
+  const uint32_t hi = __shfl_sync(0xffffffffu, static_cast<uint32_t>(x >> 32), src);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+__device__ __forceinline__ uint64_t shfl_up_u64(uint64_t x, int d) {
+  const uint32_t lo = __shfl_up_sync(0xffffffffu, static_cast<uint32_t>(x), d);
+  const uint32_t hi = __shfl_up_sync(0xffffffffu, static_cast<uint32_t>(x >> 32), d);
+  return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+__global__ void __launch_bounds__(PREP_WARPS * 32)
+prep_reg_kernel(const float* __restrict__ vals, const int32_t* __restrict__ idx, int64_t T, int K,
+                int64_t V, float inv_tau, int logprob, int32_t* __restrict__ idx_sorted,
+                float* __restrict__ p_sorted, float2* __restrict__ stats, uint32_t* status) {
+  griddep_launch_dependents();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int np = 1;
+  while (np < K) np <<= 1;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * PREP_WARPS + warp; t < T;
+       t += static_cast<int64_t>(gridDim.x) * PREP_WARPS) {
+    const float* vr = vals + t * K;
+    const int32_t* ir = idx + t * K;
+    float v[4];
+    int32_t ix[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int k = lane + 32 * r;
+      v[r] = k < K ? vr[k] : 0.f;
+      ix[r] = k < K ? ir[k] : 0;
+    }
+    float mx = 0.f, inv_se = 1.f;
+    if (!logprob) {
+      mx = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        if (lane + 32 * r < K) mx = fmaxf(mx, v[r] * inv_tau);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float se = 0.f;
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        if (lane + 32 * r < K) se += expf(v[r] * inv_tau - mx);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) se += __shfl_xor_sync(0xffffffffu, se, o);
+      inv_se = 1.f / se;
+    }
+    float S = 0.f, plogp = 0.f;
+    bool bad = false;
+    uint64_t a[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      if (lane + 32 * r < K) {
+        const float b = logprob ? v[r] : v[r] * inv_tau - mx;
+        float p = expf(b) * inv_se;
+        int32_t i = ix[r];
+        if (i < 0 || static_cast<int64_t>(i) >= V) {
+          bad = true;
+          p = 0.f;
+          i = INT32_MAX;
+        }
+        S += p;
+        if (p > 0.f) plogp += p * (logprob ? b : logf(p));
+        a[r] = (static_cast<uint64_t>(static_cast<uint32_t>(i)) << 32) | __float_as_uint(p);
+      } else {
+        a[r] = ~0ull;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      S += __shfl_xor_sync(0xffffffffu, S, o);
+      plogp += __shfl_xor_sync(0xffffffffu, plogp, o);
+    }
+    // bitonic sort of entries [0, np) ascending (the entries above np are padding)
+    for (int kk = 2; kk <= np; kk <<= 1) {
+      for (int j = kk >> 1; j > 0; j >>= 1) {
+        if (j >= 32) {
+          // entries e and e + j are this lane's registers r and r + j/32
+          auto cas = [&](uint64_t& x, uint64_t& y, int r) {
+            const bool asc = ((lane + 32 * r) & kk) == 0;
+            const bool swap = (x > y) == asc;
+            const uint64_t lo = swap ? y : x, hi = swap ? x : y;
+            x = lo;
+            y = hi;
+          };
+          if (j == 32) {
+            cas(a[0], a[1], 0);
+            cas(a[2], a[3], 2);
+          } else {
+            cas(a[0], a[2], 0);
+            cas(a[1], a[3], 1);
+          }
+        } else {
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int e = lane + 32 * r;
+            const uint64_t other = shfl_xor_u64(a[r], j);
+            const bool lower = (e & j) == 0, asc = (e & kk) == 0;
+            const bool take_min = lower == asc;
+            a[r] = take_min ? (other < a[r] ? other : a[r]) : (other > a[r] ? other : a[r]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int k = lane + 32 * r;
+      uint64_t prev = shfl_up_u64(a[r], 1);
+      const uint64_t last_prev = shfl_u64(a[r > 0 ? r - 1 : 0], 31);
+      if (lane == 0) prev = last_prev;
+      if (k < K) {
+        const uint32_t i = static_cast<uint32_t>(a[r] >> 32);
+        if (k > 0 && i != 0x7FFFFFFFu && static_cast<uint32_t>(prev >> 32) == i) bad = true;
+        idx_sorted[t * K + k] = static_cast<int32_t>(i);
+        p_sorted[t * K + k] = __uint_as_float(static_cast<uint32_t>(a[r]));
+      }
+    }
+    if (lane == 0) stats[t] = make_float2(S, plogp);
+    if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(status, KD_ERR_BAD_INDEX);
+  }
+}
+
 // ----------------------------------------------------------------------------
 // K4: combine the per-(row, vocab tile) partials of one chunk.  One warp per
 // row; lane l merges tiles l, l+32, ... in order, then a fixed shuffle tree.
@@ -312,6 +448,28 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, cu
   return cudaGetLastError();
 }
 
+// Cache preparation for fwd_impl / bwd_impl.  K <= 128: the register sort, a
+// grid small enough to be resident at once, so that the first GEMM (launched
+// with programmatic serialization) can start while it runs.  Larger K: the
+// shared-memory sort.
+cudaError_t launch_prep(const float* t_vals, const int32_t* t_idx, int64_t T, int K, int64_t V,
+                        float inv_tau, int logprob, int32_t* idx_s, float* p_s, float2* stats,
+                        uint32_t* status, cudaStream_t s, int num_sms) {
+  const int64_t blocks64 = (T + PREP_WARPS - 1) / PREP_WARPS;
+  if (K <= PREP_REG_MAXK) {
+    const int64_t cap = static_cast<int64_t>(num_sms) * 8;
+    const unsigned blocks = static_cast<unsigned>(blocks64 < cap ? blocks64 : cap);
+    prep_reg_kernel<<<blocks, PREP_WARPS * 32, 0, s>>>(t_vals, t_idx, T, K, V, inv_tau, logprob,
+                                                        idx_s, p_s, stats, status);
+  } else {
+    const int blocks = static_cast<int>(blocks64 < 65535 * 16 ? blocks64 : 65535 * 16);
+    prep_kernel<<<blocks, PREP_WARPS * 32, PREP_WARPS * PREP_MAXK * 8, s>>>(
+        t_vals, t_idx, T, K, V, inv_tau, logprob, idx_s, p_s, stats, status);
+  }
+  count_launch();
+  return cudaGetLastError();
+}
+
 // Clusters of two CTAs that can be resident at once for this kernel, cached
 // per device (atomics: calls may come from several host threads).
 constexpr int KD_MAX_DEVICES = 64;
@@ -482,15 +640,9 @@ static kd_status fwd_impl(const void* h, const void* W, int64_t T, int64_t T_nor
 
   if (cudaMemsetAsync(status, 0, 4, s) != cudaSuccess) return KD_ERR_CUDA;
   const float inv_tau = 1.f / tau;
-  {
-    const int64_t blocks64 = (T + PREP_WARPS - 1) / PREP_WARPS;
-    const int blocks = static_cast<int>(blocks64 < 65535 * 16 ? blocks64 : 65535 * 16);
-    prep_kernel<<<blocks, PREP_WARPS * 32, PREP_WARPS * PREP_MAXK * 8, s>>>(
-        t_vals, t_idx, T, K, V, inv_tau, (flags & KD_KL_LOGPROB_CACHE) ? 1 : 0, idx_s, p_s, stats,
-        status);
-    count_launch();
-    if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
-  }
+  if (launch_prep(t_vals, t_idx, T, K, V, inv_tau, (flags & KD_KL_LOGPROB_CACHE) ? 1 : 0, idx_s,
+                  p_s, stats, status, s, num_sms) != cudaSuccess)
+    return KD_ERR_CUDA;
   CUtensorMap tW;
   if (!make_map(&tW, W, F32, d, V, d, BK, 128)) return KD_ERR_CUDA;
   const float zscale = 1.4426950408889634f * inv_tau;
@@ -553,15 +705,9 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t T_nor
 
   if (cudaMemsetAsync(status, 0, 4, s) != cudaSuccess) return KD_ERR_CUDA;
   const float inv_tau = 1.f / tau;
-  {
-    const int64_t blocks64 = (T + PREP_WARPS - 1) / PREP_WARPS;
-    const int blocks = static_cast<int>(blocks64 < 65535 * 16 ? blocks64 : 65535 * 16);
-    prep_kernel<<<blocks, PREP_WARPS * 32, PREP_WARPS * PREP_MAXK * 8, s>>>(
-        t_vals, t_idx, T, K, V, inv_tau, (flags & KD_KL_LOGPROB_CACHE) ? 1 : 0, idx_s, p_s, stats,
-        status);
-    count_launch();
-    if (cudaGetLastError() != cudaSuccess) return KD_ERR_CUDA;
-  }
+  if (launch_prep(t_vals, t_idx, T, K, V, inv_tau, (flags & KD_KL_LOGPROB_CACHE) ? 1 : 0, idx_s,
+                  p_s, stats, status, s, num_sms) != cudaSuccess)
+    return KD_ERR_CUDA;
   CUtensorMap tW_k, tW_mn;
   if (!make_map(&tW_k, W, F32, d, V, d, BK, 128)) return KD_ERR_CUDA;     // [V, d], K = d
   if (!make_map(&tW_mn, W, F32, d, V, d, INNER, BK, true)) return KD_ERR_CUDA;  // K = V, N = d
