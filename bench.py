@@ -39,12 +39,12 @@ UNIT = "tokens/s"
 # 2048-row chunks at d=4096, V=131072), valid only for the GEMM sources with
 # this digest; the roofline's "traffic" is null for any other source.
 NCU_TRAFFIC = {
-    "source_sha256_16": "a7dd4ece485234b2",
+    "source_sha256_16": "99bd5f934f4ec693",
     # dram__bytes_read.sum + dram__bytes_write.sum per launch of each GEMM kind,
-    # from one capture of all 14 GEMM launches of a head-8k-c2048 step (2048-row
-    # chunks at d=4096, V=131072: the launch shapes of the 32K head); dW is the
-    # mix of a 32K step, one storing and seven accumulating launches
-    "per_launch_bytes": {"fwd_lse": 1.530e9, "bwd_dz": 2.209e9, "dH": 3.975e9, "dW": 6.570e9},
+    # from single-launch captures of a head-8k-c2048 step (2048-row chunks at
+    # d=4096, V=131072: the launch shapes of the 32K head); dW is the mix of a
+    # 32K step, one storing launch (4.791 GB) and seven adding ones (6.525 GB)
+    "per_launch_bytes": {"fwd_lse": 1.359e9, "bwd_dz": 2.101e9, "dH": 3.705e9, "dW": 6.308e9},
 }
 
 

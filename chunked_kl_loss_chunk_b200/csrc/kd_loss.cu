@@ -787,7 +787,7 @@ static kd_status bwd_impl(const void* h, const void* W, int64_t T, int64_t T_nor
       {
         const int64_t n4 = rows * (d / 4);
         int64_t blocks = (n4 + 255) / 256;
-        if (blocks > 2 * static_cast<int64_t>(num_sms)) blocks = 2 * static_cast<int64_t>(num_sms);
+        if (blocks > 4 * static_cast<int64_t>(num_sms)) blocks = 4 * static_cast<int64_t>(num_sms);
         if (launch_pdl(dh_reduce_kernel<Elem>, static_cast<unsigned>(blocks), 256u, s,
                        static_cast<const float*>(hpart), gh.k_split,
                        static_cast<int64_t>(L.rows_pad), static_cast<int>(rows), d,
