@@ -415,3 +415,29 @@ def test_peak_memory_linear_in_T():
     assert r2 > 0.999, (peaks, r2)
     assert 0.9 * expected <= b <= 1.25 * expected, (b, expected)
     assert b < 0.05 * V * 4
+
+
+def test_repeated_steps_bit_identical():
+    """The kernels of a call overlap their neighbours (programmatic dependent
+    launch) and wait inside for what those write; a missing wait would show as
+    run-to-run differences.  Many chunks (so many GEMM/combine/reduce hand-offs),
+    two dW groups with a ragged last chunk, run five times on one stream with
+    other work in between: every output bit-identical every time."""
+    require_gpu()
+    T, d, V, K, chunk = 1000, 256, 9000, 32, 96
+    h, W, vals, idx = inputs.make_loss_inputs(T, d, V, K, dtype=torch.bfloat16, seed=31, device="cuda")
+    outs = []
+    scratch = torch.empty(1 << 24, dtype=torch.float32, device="cuda")
+    for rep in range(5):
+        scratch.uniform_()                          # unrelated work on the same stream
+        loss, lse, kl, ws = kd.fused_kl_fwd(h, W, vals, idx, chunk, 1.0, kl_rows=True)
+        dH, dW, _ = kd.fused_kl_bwd(h, W, vals, idx, lse, chunk, 1.0, ws=ws)
+        torch.cuda.synchronize()
+        assert kd.read_device_status(ws) == kd.KD_OK
+        outs.append([t.clone() for t in (loss, lse, kl, dH, dW)])
+    for o in outs[1:]:
+        for a, b in zip(outs[0], o):
+            assert torch.equal(a, b)
+    hn, Wn = to_np_exact(h), to_np_exact(W)
+    lo, _, _ = oracle.forward(hn, Wn, vals.cpu().numpy(), idx.cpu().numpy(), 1.0)
+    assert abs(outs[0][0].item() - lo) <= LOSS_RTOL * abs(lo)
