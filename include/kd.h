@@ -25,6 +25,12 @@
  *     status word of its workspace when it starts.
  *   - A workspace may not be used by two calls that can run at the same time.
  *   - Device pointers must be 16-byte aligned; `ws` must be 1024-byte aligned.
+ *   - Inside one call, consecutive kernels use programmatic dependent launch:
+ *     a kernel may start while the one before it finishes, and waits inside
+ *     for that kernel's results.  The first kernel of every call is launched
+ *     in plain stream order, so a call starts only after all earlier work in
+ *     the stream; work launched after a call in plain stream order starts only
+ *     after the whole call has completed.
  */
 #ifndef KD_H_
 #define KD_H_
