@@ -9,10 +9,15 @@ with the cache the build produced feeding the loss.
 Default workload: the toy output head at 32K tokens (T=32768, d=4096,
 V=131072, K=100, chunk=2048, bf16 operands, fp32 accumulation).
 
-  python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+  python bench.py [--gpus N --steps K --warmup W] [--impl reference] [--dp]
 
-Prints ONE JSON line (rank 0).  Multi-GPU runs are independent replicas (weak
-scaling, no collective on the data path); time is the max over ranks.
+Prints ONE JSON line (rank 0).  The K timed steps are captured in one CUDA
+graph and timed as one replay, with CUDA events per step (the top-K build,
+forward and backward times) and around the GEMMs of the last step.  Multi-GPU
+runs are independent replicas by default (weak scaling, no collective on the
+data path); with --dp each rank's batch is one shard of a batch N times as
+large, and dW and the loss are summed over the ranks.  Time is the max over
+ranks.
 """
 
 from __future__ import annotations
