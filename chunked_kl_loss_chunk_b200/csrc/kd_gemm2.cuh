@@ -15,13 +15,15 @@
 // on one SM), so six stages fit and each SM pulls a third less operand data
 // through L2 per flop.
 //
-// Tiles (and, with k_split > 1, K ranges) go to clusters round-robin.  Every
+// Tiles (and, with k_split > 1, K ranges) go to clusters round-robin; each
+// role of a cluster walks its units without division (kd_unitwalk.h).  Every
 // wait is bounded; on a timeout each role leaves its loop, the leader waits for
 // the copies and MMAs it accounted for, and both CTAs meet at a cluster
 // barrier before TMEM is freed.
 #pragma once
 
 #include "kd_gemm.cuh"
+#include "kd_unitwalk.h"
 
 namespace kd {
 
@@ -127,21 +129,22 @@ __device__ __forceinline__ void mma2_commit_local(uint64_t* bar) {
       : "memory");
 }
 
-// Work unit u -> (split, m tile of 256 rows, n tile of 256 columns).
-__device__ __forceinline__ void unit_coords(const GemmArgs& g, int m_tiles2, int u, int& split,
-                                            int& mb2, int& nb) {
-  const int per_split = m_tiles2 * g.n_tiles;
-  split = u / per_split;
-  const int t = u - split * per_split;
-  mb2 = g.m_fastest ? t % m_tiles2 : t / g.n_tiles;
-  nb = g.m_fastest ? t / m_tiles2 : t % g.n_tiles;
-  KD_CHECK(split < g.k_split && mb2 < m_tiles2 && nb < g.n_tiles, g.status);
+// A cluster's walk over its work units (kd_unitwalk.h), started at unit cid.
+__device__ __forceinline__ void walk_start(UnitWalk& w, const GemmArgs& g, int m_tiles2, int cid,
+                                           int ncl) {
+  walk_begin(w, m_tiles2, g.n_tiles, g.m_fastest, g.k_blocks, g.k_split, cid, ncl);
 }
 
-// First K block of split s: the k_blocks are divided as evenly as possible,
-// so every split is non-empty when k_split <= k_blocks (the host ensures it).
-__device__ __forceinline__ int split_begin(const GemmArgs& g, int s) {
-  return static_cast<int>((static_cast<int64_t>(s) * g.k_blocks) / g.k_split);
+// Debug build: the walk's unit against its direct coordinates.
+__device__ __forceinline__ void walk_check(const UnitWalk& w, const GemmArgs& g, int m_tiles2) {
+  if (KD_DEBUG) {
+    int s, m, n;
+    unit_coords_direct(m_tiles2, g.n_tiles, g.m_fastest, w.u, s, m, n);
+    KD_CHECK(s == w.split && m == w.mb2 && n == w.nb && s < g.k_split && m < m_tiles2 &&
+                 n < g.n_tiles && w.kb0 == split_first_kblock(g.k_blocks, g.k_split, s) &&
+                 w.kb1 == split_first_kblock(g.k_blocks, g.k_split, s + 1),
+             g.status);
+  }
 }
 
 template <typename Elem, int A_MN, int B_MN, int EPI>
@@ -223,13 +226,13 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
       int stage = 0;
       uint32_t phase = 0, armed = 0, last_par = 0;
       bool ok = true;
-      for (int u = cid; ok && u < units; u += ncl) {
-        int split, mb2, nb;
-        unit_coords(g, m_tiles2, u, split, mb2, nb);
-        const int kb0 = split_begin(g, split);
-        const int kb1 = split_begin(g, split + 1);
-        const int arow = mb2 * BM2 + static_cast<int>(rank) * 128;   // this CTA's A rows
-        const int brow = nb * BN + static_cast<int>(rank) * 128;     // this CTA's B rows
+      UnitWalk w;
+      walk_start(w, g, m_tiles2, cid, ncl);
+      for (; ok && w.u < units; walk_next(w)) {
+        walk_check(w, g, m_tiles2);
+        const int kb0 = w.kb0, kb1 = w.kb1;
+        const int arow = w.mb2 * BM2 + static_cast<int>(rank) * 128;   // this CTA's A rows
+        const int brow = w.nb * BN + static_cast<int>(rank) * 128;     // this CTA's B rows
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, g.wait_limit_ns, g.status)) {
             ok = false;
@@ -281,11 +284,10 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int u = cid; ok && u < units; u += ncl) {
-        int split, mb2, nb;
-        unit_coords(g, m_tiles2, u, split, mb2, nb);
-        const int kb0 = split_begin(g, split);
-        const int kb1 = split_begin(g, split + 1);
+      UnitWalk w;
+      walk_start(w, g, m_tiles2, cid, ncl);
+      for (; ok && w.u < units; walk_next(w)) {
+        const int kb0 = w.kb0, kb1 = w.kb1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, g.wait_limit_ns, g.status)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
@@ -335,15 +337,16 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int u = cid; u < units; u += ncl) {
-      int split, mb2, nb;
-      unit_coords(g, m_tiles2, u, split, mb2, nb);
+    UnitWalk w;
+    walk_start(w, g, m_tiles2, cid, ncl);
+    for (; w.u < units; walk_next(w)) {
+      walk_check(w, g, m_tiles2);
       if (!mbar_wait(&tfull[acc], acc_phase, g.wait_limit_ns, g.status)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
-      run_epilogue<Elem, EPI>(g, &tmC, mb2 * BM2 + static_cast<int>(rank) * 128, nb, taddr, quad,
-                              lane, boxes, split * g.split_rows);
+      run_epilogue<Elem, EPI>(g, &tmC, w.mb2 * BM2 + static_cast<int>(rank) * 128, w.nb, taddr,
+                              quad, lane, boxes, w.split * g.split_rows);
       __syncwarp();
       tc_fence_before();
       if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);

@@ -37,3 +37,20 @@ def test_header_compiles_as_cxx(tmp_path):
     subprocess.run(["g++", "-std=c++17", "-Wall", "-Werror", "-I" + os.path.join(ROOT, "include"),
                     "-c", str(src), "-o", str(tmp_path / "inc.o")], check=True,
                    capture_output=True, text=True)
+
+
+def test_gemm_unit_walk_matches_direct_coordinates(tmp_path):
+    """The persistent GEMM's clusters walk their work units without division
+    (kd_unitwalk.h); on the host, the walk must give every cluster the same
+    units, tile coordinates and K ranges as the direct computation, for the
+    launch shapes of the bench workloads and for every small shape."""
+    if shutil.which("g++") is None:
+        pytest.skip("needs g++")
+    src = os.path.join(ROOT, "tests", "c", "unitwalk_check.cc")
+    exe = str(tmp_path / "unitwalk_check")
+    subprocess.run(["g++", "-std=c++17", "-O2", "-Wall", "-Werror",
+                    "-I" + os.path.join(ROOT, "chunked_kl_loss_chunk_b200", "csrc"), src, "-o", exe],
+                   check=True, capture_output=True, text=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.strip() == "ok"
