@@ -44,12 +44,13 @@ UNIT = "tokens/s"
 # 2048-row chunks at d=4096, V=131072), valid only for the GEMM sources with
 # this digest; the roofline's "traffic" is null for any other source.
 NCU_TRAFFIC = {
-    "source_sha256_16": "99bd5f934f4ec693",
+    "source_sha256_16": "dd20e58c64086fbf",
     # dram__bytes_read.sum + dram__bytes_write.sum per launch of each GEMM kind,
-    # from single-launch captures of a head-8k-c2048 step (2048-row chunks at
-    # d=4096, V=131072: the launch shapes of the 32K head); dW is the mix of a
-    # 32K step, one storing launch (4.791 GB) and seven adding ones (6.525 GB)
-    "per_launch_bytes": {"fwd_lse": 1.359e9, "bwd_dz": 2.101e9, "dH": 3.705e9, "dW": 6.308e9},
+    # from captures of one or two launches of a head-8k-c2048 step (2048-row
+    # chunks at d=4096, V=131072: the launch shapes of the 32K head); fwd_lse is
+    # the mean of two launches; dW is the mix of a 32K step, one storing launch
+    # (4.999 GB) and seven adding ones (6.662 GB)
+    "per_launch_bytes": {"fwd_lse": 1.410e9, "bwd_dz": 2.065e9, "dH": 4.154e9, "dW": 6.454e9},
 }
 
 
@@ -57,7 +58,8 @@ def _gemm_source_digest():
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "chunked_kl_loss_chunk_b200", "csrc")
-    for f in ("kd_common.cuh", "kd_gemm.cuh", "kd_gemm2.cuh", "kd_loss.cu"):
+    for f in ("kd_common.cuh", "kd_gemm.cuh", "kd_gemm2.cuh", "kd_unitwalk.h", "kd_internal.h",
+              "kd_loss.cu"):
         h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()[:16]
 
