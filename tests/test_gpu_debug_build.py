@@ -54,6 +54,9 @@ def test_debug_topk_fallback_rows(debug_lib):
     (300, 200, 5000, 16, 100, torch.bfloat16),
     (77, 72, 1003, 7, 33, torch.float32),
     (520, 264, 2304, 100, 512, torch.bfloat16),
+    # several work units per cluster (the forward and dz GEMMs: 4 x 128 tile
+    # pairs; dW: 128), so the clusters' unit walks advance under the checks
+    (1024, 256, 32768, 16, 1024, torch.bfloat16),
 ])
 def test_debug_loss_parity(debug_lib, T, d, V, K, chunk, dtype):
     h, W, vals, idx = inputs.make_loss_inputs(T, d, V, K, dtype=dtype, seed=T, device="cuda")
