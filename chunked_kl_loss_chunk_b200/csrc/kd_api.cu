@@ -129,9 +129,12 @@ kd_status kd_topk_build(const void* logits, int dtype, int64_t T, int64_t V, int
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int sms = num_sms_current();
   if (sms <= 0) return KD_ERR_CUDA;
-  if (cudaMemsetAsync(ws, 0, 4, s) != cudaSuccess) return KD_ERR_CUDA;
-  if (kd::launch_topk_bf16(logits, T, V, K, out_vals, out_idx, static_cast<uint32_t*>(ws), s,
-                           sms) != cudaSuccess)
+  // status word and row counter, both zero before the build
+  if (cudaMemsetAsync(ws, 0, kd::KD_TOPK_COUNTER_OFFSET + 8, s) != cudaSuccess) return KD_ERR_CUDA;
+  unsigned long long* row_counter = reinterpret_cast<unsigned long long*>(
+      static_cast<char*>(ws) + kd::KD_TOPK_COUNTER_OFFSET);
+  if (kd::launch_topk_bf16(logits, T, V, K, out_vals, out_idx, static_cast<uint32_t*>(ws),
+                           row_counter, s, sms) != cudaSuccess)
     return KD_ERR_CUDA;
   return KD_OK;
 }

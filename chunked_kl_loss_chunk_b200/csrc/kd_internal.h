@@ -65,8 +65,12 @@ kd_status fused_bwd(const void* h, const void* W, int dtype, int64_t T, int64_t 
                     float* dW, int accumulate, void* ws, cudaStream_t s, int num_sms,
                     uint64_t limit_ns);
 
+// The top-K build's workspace: the status word at byte 0 and the row counter
+// (zero before each build) at byte 8.
+constexpr size_t KD_TOPK_COUNTER_OFFSET = 8;
 cudaError_t launch_topk_bf16(const void* logits, int64_t T, int64_t V, int K, float* out_vals,
-                             int32_t* out_idx, uint32_t* status, cudaStream_t stream, int num_sms);
+                             int32_t* out_idx, uint32_t* status, unsigned long long* row_counter,
+                             cudaStream_t stream, int num_sms);
 
 cudaError_t launch_wait_probe(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
 

@@ -76,6 +76,7 @@ struct TopkSmem {
   uint32_t hist16[16];
   uint32_t n_cand;
   uint32_t n_sel;
+  unsigned long long row_slot[2];   // this CTA's current and next row
   uint32_t thr_bin;
   uint32_t thr_above;
   uint32_t eq_base;
@@ -436,13 +437,25 @@ __device__ __forceinline__ void stream_survivors(TopkSmem& sm, const uint16_t* _
 __global__ void __launch_bounds__(TK_THREADS, 4)
 topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int K,
                  uint32_t sample_target, int fast_sample, float* __restrict__ out_vals,
-                 int32_t* __restrict__ out_idx, uint32_t* __restrict__ status) {
+                 int32_t* __restrict__ out_idx, uint32_t* __restrict__ status,
+                 unsigned long long* __restrict__ row_counter) {
   extern __shared__ __align__(16) unsigned char tk_smem_raw[];
   TopkSmem& sm = *reinterpret_cast<TopkSmem*>(tk_smem_raw);
   const int tid = threadIdx.x;
   const bool rows_aligned = (V & 7) == 0;            // every row starts on 16 bytes
 
-  for (int64_t t = blockIdx.x; t < T; t += gridDim.x) {
+  // Rows are handed out one at a time from a counter (zero at launch): a CTA
+  // that finishes a row takes the next free one.  With a fixed share of rows
+  // per CTA the build ended when its slowest CTAs did: in one cold launch at
+  // 32768 x 131072 every CTA started at once with 55 or 56 rows, and they
+  // finished between 1.01 and 1.56 ms (the SMs do not all stream at the same
+  // rate).  A CTA takes its next row as it starts a row, so the stream's L2
+  // prefetch can run on into it.
+  if (tid == 0) sm.row_slot[0] = atomicAdd(row_counter, 1ull);
+  __syncthreads();
+  int slot = 0;
+  int64_t t_next = 0;
+  for (int64_t t = static_cast<int64_t>(sm.row_slot[0]); t < T; t = t_next, slot ^= 1) {
     const uint16_t* row = logits + t * V;
 
     // ---- 1. sample threshold -------------------------------------------------
@@ -462,8 +475,10 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
     if (tid == 0) {
       sm.n_cand = 0;
       sm.n_sel = 0;
+      sm.row_slot[slot ^ 1] = atomicAdd(row_counter, 1ull);   // read after the barrier
     }
     __syncthreads();
+    t_next = static_cast<int64_t>(sm.row_slot[slot ^ 1]);
     const uint32_t target = sample_target;
     uint32_t L;
     if (fast_sample) {
@@ -541,8 +556,8 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
 
     // ---- 2. stream the row, keep survivors ------------------------------------
     if (screen) {
-      const uint4* next_vp = (rows_aligned && t + gridDim.x < T)
-                                 ? reinterpret_cast<const uint4*>(logits + (t + gridDim.x) * V)
+      const uint4* next_vp = (rows_aligned && t_next < T)
+                                 ? reinterpret_cast<const uint4*>(logits + t_next * V)
                                  : nullptr;
       stream_survivors(sm, row, static_cast<uint32_t>(V), tf, next_vp, status);
     }
@@ -808,7 +823,8 @@ topk_bf16_kernel(const uint16_t* __restrict__ logits, int64_t T, int64_t V, int 
 namespace kd {
 
 cudaError_t launch_topk_bf16(const void* logits, int64_t T, int64_t V, int K, float* out_vals,
-                             int32_t* out_idx, uint32_t* status, cudaStream_t stream, int num_sms) {
+                             int32_t* out_idx, uint32_t* status, unsigned long long* row_counter,
+                             cudaStream_t stream, int num_sms) {
   const size_t smem = sizeof(TopkSmem);
   cudaError_t e = cudaFuncSetAttribute(topk_bf16_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -834,7 +850,8 @@ cudaError_t launch_topk_bf16(const void* logits, int64_t T, int64_t V, int K, fl
   // long and 16-byte aligned and the target is a small share of the 256 keys
   const int fast = (V > TK_SAMPLE && (V & 7) == 0 && target <= 32u) ? 1 : 0;
   topk_bf16_kernel<<<static_cast<unsigned>(grid), TK_THREADS, smem, stream>>>(
-      static_cast<const uint16_t*>(logits), T, V, K, target, fast, out_vals, out_idx, status);
+      static_cast<const uint16_t*>(logits), T, V, K, target, fast, out_vals, out_idx, status,
+      row_counter);
   count_launch();
   return cudaGetLastError();
 }

@@ -70,7 +70,8 @@ int kd_version(void);
 /* the teacher is run once and its top-K tokens per position are cached.    */
 /* ------------------------------------------------------------------------ */
 
-/* Bytes of workspace kd_topk_build needs (the device status word). */
+/* Bytes of workspace kd_topk_build needs (the device status word and the
+ * counter that hands rows to the kernel's thread blocks). */
 size_t kd_topk_workspace_size(int64_t T, int64_t V, int K);
 
 /*
@@ -82,9 +83,12 @@ size_t kd_topk_workspace_size(int64_t T, int64_t V, int K);
  *   out_idx  int32   [T, K]: their column indices.
  * Requires 1 <= K <= min(V, 1024), T >= 1, V < 2^31.
  * ws (1024-byte aligned, ws_bytes >= kd_topk_workspace_size) holds the
- * device status word, cleared at the start of the call; only the debug build
- * records anything there (KD_ERR_INTERNAL).  Read it with
- * kd_read_device_status.
+ * device status word and a row counter, both cleared at the start of the
+ * call; only the debug build records anything in the status word
+ * (KD_ERR_INTERNAL).  Read it with kd_read_device_status.  Rows go to the
+ * kernel's thread blocks in the order they ask for them, so the workspace must
+ * not be shared with a build running at the same time; each row's result does
+ * not depend on which block computed it.
  */
 kd_status kd_topk_build(const void* logits, int dtype, int64_t T, int64_t V, int K,
                         float* out_vals, int32_t* out_idx,
