@@ -44,13 +44,13 @@ UNIT = "tokens/s"
 # 2048-row chunks at d=4096, V=131072), valid only for the GEMM sources with
 # this digest; the roofline's "traffic" is null for any other source.
 NCU_TRAFFIC = {
-    "source_sha256_16": "dd20e58c64086fbf",
+    "source_sha256_16": "66c94b05b3f692c4",
     # dram__bytes_read.sum + dram__bytes_write.sum per launch of each GEMM kind,
     # from captures of one or two launches of a head-8k-c2048 step (2048-row
     # chunks at d=4096, V=131072: the launch shapes of the 32K head); fwd_lse is
     # the mean of two launches; dW is the mix of a 32K step, one storing launch
-    # (4.999 GB) and seven adding ones (6.662 GB)
-    "per_launch_bytes": {"fwd_lse": 1.410e9, "bwd_dz": 2.065e9, "dH": 4.154e9, "dW": 6.454e9},
+    # (4.468 GB) and seven adding ones (5.905 GB)
+    "per_launch_bytes": {"fwd_lse": 1.168e9, "bwd_dz": 1.790e9, "dH": 3.186e9, "dW": 5.726e9},
 }
 
 
