@@ -149,9 +149,12 @@ __device__ __forceinline__ int lower_bound_i32(const int32_t* ids, int K, int32_
 // of tcgen05.ld (they are warp-collective).
 // ----------------------------------------------------------------------------
 template <typename Elem, int EPI>
+// pace_ns (EPI_ACCUM_W): pause between two output boxes of a warp, so that a
+// tile's fp32 dW boxes go out spread over the next tile's mainloop.
 __device__ __forceinline__ void run_epilogue(const GemmArgs& g, const CUtensorMap* tmC, int m_base,
                                              int nb, uint32_t taddr, int quad, int lane,
-                                             unsigned char* boxes, int y_extra = 0) {
+                                             unsigned char* boxes, int y_extra = 0,
+                                             uint32_t pace_ns = 0) {
   const int r = quad * 32 + lane;         // accumulator row of this thread
   const int m = m_base + r;               // output row within the problem
   const bool row_ok = m < g.M;
@@ -257,6 +260,7 @@ __device__ __forceinline__ void run_epilogue(const GemmArgs& g, const CUtensorMa
       if constexpr (EPI == EPI_STORE_H && sizeof(Elem) == 2) stage_box_bf16(box, lane, v);
       else stage_box_f32(box, lane, v);
       emit_box<Elem>(tmC, box, base, y_box, EPI == EPI_ACCUM_W && g.accumulate);
+      if (EPI == EPI_ACCUM_W && pace_ns) __nanosleep(pace_ns);
     }
   }
 }

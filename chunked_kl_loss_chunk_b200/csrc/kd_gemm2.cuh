@@ -337,16 +337,37 @@ gemm2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CU
     const uint32_t tempty_leader1 = mapa_shared(smem_u32(&tempty[1]), 0);
     int acc = 0;
     uint32_t acc_phase = 0;
+    // dW: every cluster finishes its tiles at about the same moment, and each
+    // CTA then adds 128 KB of fp32 into dW.  Sent as one burst, the add-
+    // reductions of all clusters crowd out the operand loads of the next
+    // tiles, and the MMAs wait for data (measured: the issue span of a dW tile
+    // was 0.93 of its ideal tensor time, 0.99 with the boxes spread).  So the
+    // epilogue spaces its boxes by 1/16 of the time between two of its tiles
+    // (the tiles before), which spreads them over about half of the next
+    // tile's mainloop at any clock.
+    uint64_t prev_ready = 0;
+    uint32_t pace_ns = 0;
     UnitWalk w;
     walk_start(w, g, m_tiles2, cid, ncl);
     for (; w.u < units; walk_next(w)) {
       walk_check(w, g, m_tiles2);
       if (!mbar_wait(&tfull[acc], acc_phase, g.wait_limit_ns, g.status)) break;
       tc_fence_after();
+      if (EPI == EPI_ACCUM_W) {
+        if (lane == 0) {
+          const uint64_t now = globaltimer_ns();
+          if (prev_ready != 0) {
+            const uint64_t p = (now - prev_ready) / (2 * (BN / 32));
+            pace_ns = static_cast<uint32_t>(p < 4000 ? p : 4000);
+          }
+          prev_ready = now;
+        }
+        pace_ns = __shfl_sync(0xffffffffu, pace_ns, 0);
+      }
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                              static_cast<uint32_t>(acc * BN);
       run_epilogue<Elem, EPI>(g, &tmC, w.mb2 * BM2 + static_cast<int>(rank) * 128, w.nb, taddr,
-                              quad, lane, boxes, w.split * g.split_rows);
+                              quad, lane, boxes, w.split * g.split_rows, pace_ns);
       __syncwarp();
       tc_fence_before();
       if (lane == 0) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
