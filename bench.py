@@ -44,13 +44,13 @@ UNIT = "tokens/s"
 # 2048-row chunks at d=4096, V=131072), valid only for the GEMM sources with
 # this digest; the roofline's "traffic" is null for any other source.
 NCU_TRAFFIC = {
-    "source_sha256_16": "66c94b05b3f692c4",
+    "source_sha256_16": "0ec119d57cec7fff",
     # dram__bytes_read.sum + dram__bytes_write.sum per launch of each GEMM kind,
     # from captures of one or two launches of a head-8k-c2048 step (2048-row
     # chunks at d=4096, V=131072: the launch shapes of the 32K head); fwd_lse is
     # the mean of two launches; dW is the mix of a 32K step, one storing launch
-    # (4.468 GB) and seven adding ones (5.905 GB)
-    "per_launch_bytes": {"fwd_lse": 1.168e9, "bwd_dz": 1.790e9, "dH": 3.186e9, "dW": 5.726e9},
+    # (4.075 GB) and seven adding ones (5.833 GB)
+    "per_launch_bytes": {"fwd_lse": 1.112e9, "bwd_dz": 1.630e9, "dH": 2.617e9, "dW": 5.613e9},
 }
 
 
