@@ -282,6 +282,7 @@ class ClockSampler:
             ident = "GPU-" + str(u) if not str(u).startswith("GPU-") else str(u)
         except Exception:
             pass
+        self.ident = ident
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
@@ -299,25 +300,53 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in open(self.path):
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
+        result = parse_clock_samples(open(self.path).read().splitlines())
         os.unlink(self.path)
-        if not sm:
+        if result is not None:
+            result["power_limit_w"] = self.power_limit()
+        return result
+
+    def power_limit(self):
+        """The board's enforced power limit in watts (one nvidia-smi query;
+        None if it cannot be read)."""
+        try:
+            out = subprocess.run(["nvidia-smi", f"--id={self.ident}",
+                                  "--query-gpu=enforced.power.limit",
+                                  "--format=csv,noheader,nounits"],
+                                 capture_output=True, text=True, timeout=10).stdout
+            return float(out.strip().splitlines()[0])
+        except Exception:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+
+
+def parse_clock_samples(lines):
+    """nvidia-smi CSV lines (index, clocks.sm, clocks.max.sm, power.draw, the
+    active-reasons bitmask, then hw_slowdown, hw_thermal_slowdown,
+    sw_thermal_slowdown, sw_power_cap) -> the median SM clock, the highest max
+    clock, every reason seen active, the median board power and the number of
+    samples; None without a parsable line."""
+    sm, mx, pw, reasons = [], [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for ln in lines:
+        f = [x.strip() for x in ln.split(",")]
+        if len(f) < 9:
+            continue
+        try:
+            sm.append(float(f[1]))
+            mx.append(float(f[2]))
+        except ValueError:
+            continue
+        try:
+            pw.append(float(f[3]))
+        except ValueError:
+            pass
+        for n, v in zip(names, f[5:9]):
+            if v.lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return None
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+            "power_w": statistics.median(pw) if pw else None, "samples": len(sm)}
 
 
 # ------------------------------------------------------------------ GPU arm
@@ -674,6 +703,12 @@ def run_kd(args, rank, world):
                      "peak_source": f"{peak_src} bf16_tflops_sustained (kernel inside a long step)"},
         "gpu_launches": int(n_launch),
         "clocks": clocks,
+        # board power sampled during the timed steps (rank 0's GPU): the
+        # energy of one step, and the step's 8TdV flops per joule of it
+        "energy": (None if not clocks or clocks.get("power_w") is None else {
+            "power_w_median": clocks["power_w"],
+            "joules_per_step": clocks["power_w"] * ms_step / 1e3,
+            "tflop_per_joule": flop_step / 1e12 / (clocks["power_w"] * ms_step / 1e3)}),
         "e2e": e2e,
         "cpu_baseline": cpu,
     }

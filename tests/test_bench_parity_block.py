@@ -52,3 +52,19 @@ def test_planted_mistakes_fail():
     bad["dH"][sel[-1]] *= 1.05
     p = _parity(bad, w)
     assert p["dH_rel_maxabs_err"] > 2e-2 and not p["pass"]
+
+
+def test_clock_samples_parse_power_and_reasons():
+    """The bench's nvidia-smi sampler: median SM clock and board power, the
+    highest max clock, every throttle reason seen active; unparsable power
+    fields are skipped, malformed lines ignored, no samples give None."""
+    import bench
+    lines = ["0, 1350, 1965, 998.50, 0x4, Not Active, Not Active, Not Active, Active",
+             "0, 1365, 1965, 1001.20, 0x4, Not Active, Not Active, Not Active, Active",
+             "0, 1290, 1965, [N/A], 0x4, Active, Not Active, Not Active, Not Active",
+             "no, data"]
+    r = bench.parse_clock_samples(lines)
+    assert r["sm_mhz"] == 1350.0 and r["sm_max_mhz"] == 1965.0 and r["samples"] == 3
+    assert r["power_w"] == (998.50 + 1001.20) / 2
+    assert r["reasons"] == ["hw_slowdown", "sw_power_cap"]
+    assert bench.parse_clock_samples(["garbage"]) is None
