@@ -5,18 +5,24 @@
 // Per row of bf16 teacher logits, select the K entries ranked by
 // (value descending, index ascending), +0 == -0, NaN below -inf.
 //
-// Design (HBM-bound streaming select):
-//   1. sample: a 4096-bin histogram (order key >> 4) of the first
-//      min(V, 4096) elements, refined inside the threshold bin, gives the key L
-//      of the sample element ranked ~3K*S/V from the top (about 3K expected
-//      survivors in the row).  L is turned into a float threshold tf with
+// Design (HBM-bound streaming select).  Four 256-thread blocks per SM; each
+// takes one row at a time from a counter in the workspace:
+//   1. sample: the key L of the sample element ranked about 3K*S/V from the
+//      top of the row's first S = min(V, 4096) elements (about 3K expected
+//      survivors in the row), found in two levels of 256 bins (the key's high
+//      byte, then its low byte).  On long aligned rows each thread contributes
+//      the largest of its 16 sample elements instead (a packed bf16 maximum),
+//      which can only lower L.  L is turned into a bf16 threshold tf with
 //      key(x) >= L  <=>  x >= tf  for every non-NaN x.
-//   2. stream: one coalesced 16-byte-vector pass over the row; each element is
-//      one float compare against tf; the rare survivors are appended to a
-//      shared-memory candidate buffer.
+//   2. stream: one coalesced pass over the row with eight 16-byte loads in
+//      flight per thread; each vector is screened by its packed maximum, the
+//      warp stages the vectors that may hold a survivor and tests them element
+//      by element, and the survivors are appended to a shared-memory buffer.
+//      One thread keeps the stream two steps ahead in L2, into the next row.
 //   3. if K <= survivors <= capacity, the top K of the row are exactly the top
-//      K of the survivors: bitonic-sort them by the composite (key desc,
-//      index asc) and write the first K.
+//      K of the survivors, ordered by the composite (key desc, index asc):
+//      usually through one 256-bin histogram of key - L, otherwise by a wider
+//      histogram and counting.
 //   4. otherwise (ties, NaN-heavy or adversarially ordered rows) an exact
 //      3-pass histogram select runs instead (passes 2-3 hit L2).
 #include "kd_common.cuh"
